@@ -1,0 +1,624 @@
+/*
+ * ecco_oracle.c -- plain, slow, obviously-correct CPU oracle for the Ecco
+ * 512-bit block codec.  TEST INFRASTRUCTURE ONLY: tests/, the smoke check and
+ * the CPU-baseline leg of bench.py may call it; the product path never does.
+ *
+ * Source method: "Ecco: Improving Memory Bandwidth and Capacity for LLMs via
+ * Entropy-aware Cache Compression" (arXiv 2505.06901), as summarised on its
+ * pith.science review page.  Passages followed, by section of that page:
+ *   - "What carries the argument": 128-value groups, 64 shared patterns of 15
+ *     sorted centroids, 4 Huffman codebooks per pattern chosen by shortest
+ *     length, clipping of overflow, padding with the largest remaining
+ *     outliers, fixed 512-bit block, min/max pattern selection.
+ *   - "Core claim": per-group FP8 scale, overflow clipped, spare space padded
+ *     with the next-largest outliers.
+ *   - Fig. 4 caption: per-tensor FP16-to-FP8 scale factor; the normalised FP8
+ *     value is the group scale; values normalised to (-1, 1).
+ *   - Free parameters: "index 15 reserved for the scale factor"; "Top-16 values
+ *     ... up to 240 bits per block"; block size 64 bytes; min/max squared error.
+ *   - Referee major comment 1 (Sec. 4.2, Fig. 8): code lengths limited to 2-8 bits.
+ *   - Circularity check (Sec. 3.1 / 3.2 step 9): "If the compressed data exceeds
+ *     the block size, we simply clip the excess."
+ *
+ * Where the page is silent the oracle follows these readings (each one is a
+ * line of the format specification that the CUDA path implements too):
+ *   R1  bit order: stream bit b is bit (b%8) of byte b/8 (little-endian words).
+ *       A codeword is emitted most-significant code bit first.
+ *   R2  header: bits 0-7 FP8 E4M3 scale code, 8-13 pattern p, 14-15 codebook h.
+ *       Payload bits 16..511.
+ *   R3  S_t is a table input (fp32).
+ *   R4  m = first index of max |x| (bf16 magnitude); r = x_m / S_t (fp32);
+ *       code = E4M3(r) round-half-even, saturating to +-448; s = S_t * fp8(code)
+ *       (fp32), signed.
+ *   R5  element m gets symbol 15, reconstructed as exactly s.
+ *   R6  inv = 1/s (fp32 IEEE), u_i = x_i * inv (fp32).
+ *   R7  fp8(code) == 0  ->  the whole block is 64 zero bytes.
+ *   R8  e_p = (umin - C[p][0])^2 + (umax - C[p][14])^2 over i != m, every op
+ *       rounded to fp32 separately; first p with the least e_p.
+ *   R9  sym = #{ j in 0..13 : u > T[p][j] }, T[p][j] = (C[p][j] + C[p][j+1]) * 0.5.
+ *   R11 code lengths 1..8, complete (Kraft sum exactly 1).
+ *   R12 canonical codes by (length, symbol) ascending.
+ *   R13 h = first codebook with the least total length of the 128 codewords.
+ *   R14 codewords in index order; the first one that does not fit is written
+ *       up to bit 511 and nothing after it; decoded elements from there on are +0.
+ *   R15 unclipped blocks with L payload bits carry n = min(16, (496-L)/15)
+ *       records of 7-bit position then 8-bit q = clamp(rint(u*127), -127, 127);
+ *       decoded as bf16(s * (q / 127)).
+ *   R16 record candidates are i != m ranked by |x_i| descending, ties by index.
+ *   R17 decoded value = bf16 round-half-even of fp32(s * C[p][sym]).
+ *   R18 scale codes 0x00, 0x80 (zero) and 0x7f, 0xff (NaN) decode to 128 x +0;
+ *       records are applied in order (last wins).
+ *   R21 a NaN or +-Inf input element is encoded as +0.0 and counted.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC -pthread.
+ * Shares no source with the CUDA library.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_G 128
+#define OR_NPAT 64
+#define OR_NCENT 15
+#define OR_NBOOK 4
+#define OR_NSYM 16
+#define OR_LMAX 8
+#define OR_BLOCK_BYTES 64
+#define OR_BLOCK_BITS 512
+#define OR_HDR_BITS 16
+#define OR_PAYLOAD_BITS 496
+#define OR_REC_BITS 15
+#define OR_MAX_REC 16
+#define OR_MAGIC 0x31434345u /* "ECC1" little-endian */
+
+/* Table blob, as handed to both implementations (a file format, little-endian). */
+typedef struct {
+    uint32_t magic;
+    uint32_t version;
+    float S_t;
+    uint32_t reserved;
+    float C[OR_NPAT][OR_NCENT];
+    uint8_t len[OR_NPAT][OR_NBOOK][OR_NSYM];
+} or_tables;
+
+typedef struct {
+    uint64_t n_groups;
+    uint64_t n_zero;
+    uint64_t n_clipped;
+    uint64_t n_padded;      /* unclipped blocks carrying >= 1 record */
+    uint64_t n_records;
+    uint64_t n_nonfinite;
+    uint64_t payload_bits;  /* sum of min(L, 496) over non-zero blocks */
+    uint64_t n_mse_differs; /* groups whose full-MSE pattern differs from min/max */
+    double mse_minmax;      /* sum of squared normalised error, min/max choice */
+    double mse_full;        /* same with the full-MSE choice */
+} or_stats;
+
+/* Everything the encoder decided for one group (for step-by-step tests). */
+typedef struct {
+    int32_t m;
+    int32_t zero;
+    uint8_t code;
+    uint8_t p;
+    uint8_t h;
+    uint8_t clipped;
+    float s;
+    float inv;
+    float umin;
+    float umax;
+    int32_t L;      /* total payload bits of the 128 codewords, unclipped length */
+    int32_t k_clip; /* first element not fully written (128 if none) */
+    int32_t n_rec;
+    uint8_t sym[OR_G];
+    uint8_t rec_pos[OR_MAX_REC];
+    int8_t rec_q[OR_MAX_REC];
+    float u[OR_G];  /* u[m] is left as 0 */
+    float e[OR_NPAT];
+    int32_t Lh[OR_NBOOK];
+    int32_t nonfinite;
+} or_group_info;
+
+/* ------------------------------------------------------------------ */
+/* Number formats, from their public definitions.                      */
+/* ------------------------------------------------------------------ */
+
+static float f32_from_bits(uint32_t b) { float f; memcpy(&f, &b, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t b; memcpy(&b, &f, 4); return b; }
+
+/* bf16 is the top half of an IEEE binary32. */
+float or_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* IEEE round-to-nearest, ties to even, binary32 -> bfloat16.  NaN -> 0x7fc0|sign. */
+uint16_t or_f32_to_bf16(float f)
+{
+    uint32_t u = bits_from_f32(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)(((u >> 16) & 0x8000u) | 0x7fc0u);
+    uint32_t upper = u >> 16;
+    uint32_t lower = u & 0xffffu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u; /* may carry into Inf */
+    return (uint16_t)upper;
+}
+
+/* OCP 8-bit floating point, E4M3: bias 7, no infinities, S.1111.111 is NaN,
+ * subnormals m * 2^-9.  Returns the exact value as a double. */
+double or_e4m3_value(uint8_t c)
+{
+    int sgn = (c >> 7) & 1;
+    int e = (c >> 3) & 15;
+    int m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* Round a finite binary32 to E4M3 by brute force: the nearest of the 127
+ * non-negative finite codes, ties to the even code (even mantissa), values
+ * at or beyond the largest finite (448) saturate to it.  The sign is copied. */
+uint8_t or_e4m3_from_f32(float r)
+{
+    double a = fabs((double)r);
+    uint8_t best = 0;
+    double bestd = INFINITY;
+    if (a >= 448.0) best = 0x7e;
+    else {
+        for (int c = 0; c <= 0x7e; ++c) {
+            double d = fabs(a - or_e4m3_value((uint8_t)c));
+            if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+                bestd = d;
+                best = (uint8_t)c;
+            }
+        }
+    }
+    return (uint8_t)(best | (signbit(r) ? 0x80 : 0x00));
+}
+
+/* ------------------------------------------------------------------ */
+/* Tables                                                              */
+/* ------------------------------------------------------------------ */
+
+/* Returns 0 if the blob is a valid table set, else a negative reason code. */
+int or_tables_check(const or_tables* t)
+{
+    if (t->magic != OR_MAGIC || t->version != 1u) return -1;
+    float st = t->S_t;
+    if (!isfinite(st) || !(st >= ldexpf(1.0f, -60)) || !(st <= ldexpf(1.0f, 60))) return -2;
+    for (int p = 0; p < OR_NPAT; ++p)
+        for (int j = 0; j < OR_NCENT; ++j) {
+            float c = t->C[p][j];
+            if (!isfinite(c) || fabsf(c) > 4.0f) return -3;
+            if (j > 0 && !(t->C[p][j - 1] < c)) return -4;
+        }
+    for (int p = 0; p < OR_NPAT; ++p)
+        for (int h = 0; h < OR_NBOOK; ++h) {
+            uint32_t kraft = 0; /* in units of 2^-8 */
+            for (int s = 0; s < OR_NSYM; ++s) {
+                int l = t->len[p][h][s];
+                if (l < 1 || l > OR_LMAX) return -5;
+                kraft += 1u << (OR_LMAX - l);
+            }
+            if (kraft != (1u << OR_LMAX)) return -6;
+        }
+    return 0;
+}
+
+/* Canonical code of one codebook: symbols ordered by (length, symbol); the
+ * first gets code 0, each next one (previous + 1) shifted left by the length
+ * increase. */
+static void canonical_codes(const uint8_t len[OR_NSYM], uint32_t code[OR_NSYM])
+{
+    int order[OR_NSYM];
+    int n = 0;
+    for (int l = 1; l <= OR_LMAX; ++l)
+        for (int s = 0; s < OR_NSYM; ++s)
+            if (len[s] == l) order[n++] = s;
+    uint32_t c = 0;
+    for (int i = 0; i < n; ++i) {
+        int s = order[i];
+        if (i > 0) c = (c + 1u) << (len[s] - len[order[i - 1]]);
+        code[s] = c;
+    }
+}
+
+void or_canonical_codes(const or_tables* t, int p, int h, uint32_t* code_out)
+{
+    canonical_codes(t->len[p][h], code_out);
+}
+
+static float threshold(const or_tables* t, int p, int j)
+{
+    float sum = t->C[p][j] + t->C[p][j + 1];
+    return sum * 0.5f;
+}
+
+/* ------------------------------------------------------------------ */
+/* Bit stream                                                          */
+/* ------------------------------------------------------------------ */
+
+static void put_bit(uint8_t* blk, int pos, int bit)
+{
+    if (pos < OR_BLOCK_BITS && bit) blk[pos >> 3] |= (uint8_t)(1u << (pos & 7));
+}
+
+static int get_bit(const uint8_t* blk, int pos) { return (blk[pos >> 3] >> (pos & 7)) & 1; }
+
+/* Writes `nbits` of `value`, least-significant bit first, from `pos`. */
+static void put_field(uint8_t* blk, int pos, uint32_t value, int nbits)
+{
+    for (int i = 0; i < nbits; ++i) put_bit(blk, pos + i, (value >> i) & 1u);
+}
+
+static uint32_t get_field(const uint8_t* blk, int pos, int nbits)
+{
+    uint32_t v = 0;
+    for (int i = 0; i < nbits; ++i) v |= (uint32_t)get_bit(blk, pos + i) << i;
+    return v;
+}
+
+/* Writes a codeword most-significant bit first; bits past 511 are dropped. */
+static void put_codeword(uint8_t* blk, int pos, uint32_t code, int len)
+{
+    for (int i = 0; i < len; ++i) put_bit(blk, pos + i, (code >> (len - 1 - i)) & 1u);
+}
+
+/* ------------------------------------------------------------------ */
+/* Encoder: one group of 128 bf16 values -> one 64-byte block          */
+/* ------------------------------------------------------------------ */
+
+static int quantise(const or_tables* t, int p, float u)
+{
+    int sym = 0;
+    for (int j = 0; j < OR_NCENT - 1; ++j)
+        if (u > threshold(t, p, j)) sym += 1;
+    return sym;
+}
+
+/* Full squared error of the normalised group under pattern p (fp64 sum). */
+static double pattern_mse(const or_tables* t, int p, const float* u, int m)
+{
+    double acc = 0.0;
+    for (int i = 0; i < OR_G; ++i) {
+        if (i == m) continue;
+        double d = (double)u[i] - (double)t->C[p][quantise(t, p, u[i])];
+        acc += d * d;
+    }
+    return acc;
+}
+
+/* force_p / force_h < 0: the method's own choice; >= 0: forced (tests only). */
+void or_encode_group_ex(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
+                        or_group_info* info, int force_p, int force_h)
+{
+    or_group_info gi;
+    memset(&gi, 0, sizeof gi);
+    memset(blk, 0, OR_BLOCK_BYTES);
+
+    /* R21: non-finite elements become +0. */
+    uint16_t x[OR_G];
+    for (int i = 0; i < OR_G; ++i) {
+        x[i] = x_in[i];
+        if ((x[i] & 0x7f80u) == 0x7f80u) { x[i] = 0; gi.nonfinite += 1; }
+    }
+
+    /* R4: first index of the largest magnitude. */
+    int m = 0;
+    for (int i = 1; i < OR_G; ++i)
+        if ((x[i] & 0x7fffu) > (x[m] & 0x7fffu)) m = i;
+    gi.m = m;
+
+    float xm = or_bf16_to_f32(x[m]);
+    float r = xm / t->S_t;
+    uint8_t code = or_e4m3_from_f32(r);
+    double fp8v = or_e4m3_value(code);
+    gi.code = code;
+    gi.k_clip = OR_G;
+    if (fp8v == 0.0) { /* R7 */
+        gi.zero = 1;
+        gi.code = 0;
+        for (int i = 0; i < OR_G; ++i) gi.sym[i] = 0;
+        if (info) *info = gi;
+        return;
+    }
+    float s = t->S_t * (float)fp8v;
+    float inv = 1.0f / s;
+    gi.s = s;
+    gi.inv = inv;
+
+    /* R6 */
+    float u[OR_G];
+    for (int i = 0; i < OR_G; ++i) u[i] = (i == m) ? 0.0f : or_bf16_to_f32(x[i]) * inv;
+    memcpy(gi.u, u, sizeof u);
+
+    /* R8: min/max pattern fitness. */
+    float umin = INFINITY, umax = -INFINITY;
+    for (int i = 0; i < OR_G; ++i) {
+        if (i == m) continue;
+        if (u[i] < umin) umin = u[i];
+        if (u[i] > umax) umax = u[i];
+    }
+    gi.umin = umin;
+    gi.umax = umax;
+    int p = 0;
+    for (int q = 0; q < OR_NPAT; ++q) {
+        float d0 = umin - t->C[q][0];
+        float d1 = umax - t->C[q][OR_NCENT - 1];
+        float sq0 = d0 * d0;
+        float sq1 = d1 * d1;
+        float e = sq0 + sq1;
+        gi.e[q] = e;
+        if (e < gi.e[p]) p = q;
+    }
+    if (force_p >= 0) p = force_p;
+    gi.p = (uint8_t)p;
+
+    /* R5, R9 */
+    for (int i = 0; i < OR_G; ++i) gi.sym[i] = (uint8_t)((i == m) ? 15 : quantise(t, p, u[i]));
+
+    /* R13: shortest codebook over the whole group. */
+    int h = 0;
+    for (int b = 0; b < OR_NBOOK; ++b) {
+        int L = 0;
+        for (int i = 0; i < OR_G; ++i) L += t->len[p][b][gi.sym[i]];
+        gi.Lh[b] = L;
+        if (L < gi.Lh[h]) h = b;
+    }
+    if (force_h >= 0) h = force_h;
+    gi.h = (uint8_t)h;
+
+    /* R2 header */
+    put_field(blk, 0, code, 8);
+    put_field(blk, 8, (uint32_t)p, 6);
+    put_field(blk, 14, (uint32_t)h, 2);
+
+    /* R1, R12, R14: pack codewords, clip at bit 512. */
+    uint32_t cw[OR_NSYM];
+    canonical_codes(t->len[p][h], cw);
+    int pos = OR_HDR_BITS;
+    int L = 0;
+    for (int i = 0; i < OR_G; ++i) {
+        int l = t->len[p][h][gi.sym[i]];
+        if (pos + l > OR_BLOCK_BITS && gi.k_clip == OR_G) gi.k_clip = i;
+        if (pos < OR_BLOCK_BITS) put_codeword(blk, pos, cw[gi.sym[i]], l);
+        pos += l;
+        L += l;
+    }
+    gi.L = L;
+    gi.clipped = (gi.k_clip < OR_G);
+
+    /* R15, R16: outlier records in the spare bits. */
+    if (!gi.clipped) {
+        int n = (OR_PAYLOAD_BITS - L) / OR_REC_BITS;
+        if (n > OR_MAX_REC) n = OR_MAX_REC;
+        uint8_t taken[OR_G];
+        memset(taken, 0, sizeof taken);
+        taken[m] = 1;
+        for (int k = 0; k < n; ++k) {
+            int best = -1;
+            for (int i = 0; i < OR_G; ++i) {
+                if (taken[i]) continue;
+                if (best < 0 || (x[i] & 0x7fffu) > (x[best] & 0x7fffu)) best = i;
+            }
+            taken[best] = 1;
+            float v = u[best] * 127.0f;
+            float rq = rintf(v);
+            if (rq > 127.0f) rq = 127.0f;
+            if (rq < -127.0f) rq = -127.0f;
+            int q = (int)rq;
+            gi.rec_pos[k] = (uint8_t)best;
+            gi.rec_q[k] = (int8_t)q;
+            int at = OR_HDR_BITS + L + k * OR_REC_BITS;
+            put_field(blk, at, (uint32_t)best, 7);
+            put_field(blk, at + 7, (uint32_t)(uint8_t)(int8_t)q, 8);
+        }
+        gi.n_rec = n;
+    }
+    if (info) *info = gi;
+}
+
+void or_encode_group(const or_tables* t, const uint16_t* x, uint8_t* blk, or_group_info* info)
+{
+    or_encode_group_ex(t, x, blk, info, -1, -1);
+}
+
+/* ------------------------------------------------------------------ */
+/* Decoder: one 64-byte block -> 128 bf16 values                        */
+/* ------------------------------------------------------------------ */
+
+/* Reads one codeword bit by bit; returns the symbol, or -1 if the block ends first. */
+static int read_codeword(const uint8_t* blk, int* pos, const uint8_t len[OR_NSYM],
+                         const uint32_t code[OR_NSYM])
+{
+    uint32_t acc = 0;
+    for (int l = 1; l <= OR_LMAX; ++l) {
+        if (*pos + l > OR_BLOCK_BITS) return -1;
+        acc = (acc << 1) | (uint32_t)get_bit(blk, *pos + l - 1);
+        for (int s = 0; s < OR_NSYM; ++s)
+            if (len[s] == l && code[s] == acc) { *pos += l; return s; }
+    }
+    return -1; /* unreachable for a complete code */
+}
+
+/* Returns the number of elements decoded from codewords (128 unless clipped). */
+int or_decode_block(const or_tables* t, const uint8_t* blk, uint16_t* y)
+{
+    for (int i = 0; i < OR_G; ++i) y[i] = 0;
+    uint8_t code = (uint8_t)get_field(blk, 0, 8);
+    int p = (int)get_field(blk, 8, 6);
+    int h = (int)get_field(blk, 14, 2);
+    double fp8v = or_e4m3_value(code);
+    if (isnan(fp8v) || fp8v == 0.0) return 0; /* R7, R18 */
+    float s = t->S_t * (float)fp8v;
+
+    uint32_t cw[OR_NSYM];
+    canonical_codes(t->len[p][h], cw);
+    int pos = OR_HDR_BITS;
+    int k = 0;
+    for (; k < OR_G; ++k) {
+        int sym = read_codeword(blk, &pos, t->len[p][h], cw);
+        if (sym < 0) break;
+        float c = (sym == 15) ? 1.0f : t->C[p][sym];
+        y[k] = or_f32_to_bf16(s * c);
+    }
+    if (k == OR_G) {
+        int L = pos - OR_HDR_BITS;
+        int n = (OR_PAYLOAD_BITS - L) / OR_REC_BITS;
+        if (n > OR_MAX_REC) n = OR_MAX_REC;
+        for (int r = 0; r < n; ++r) {
+            int at = pos + r * OR_REC_BITS;
+            int i = (int)get_field(blk, at, 7);
+            int q = (int)(int8_t)(uint8_t)get_field(blk, at + 7, 8);
+            float o = (float)q / 127.0f;
+            y[i] = or_f32_to_bf16(s * o);
+        }
+    }
+    return k;
+}
+
+/* ------------------------------------------------------------------ */
+/* Whole arrays (groups are independent; threads split the group range) */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const or_tables* t;
+    const uint16_t* x;
+    uint8_t* blocks;
+    uint16_t* y;
+    int64_t lo, hi;
+    int with_mse;
+    or_stats st;
+} or_job;
+
+static void* encode_worker(void* arg)
+{
+    or_job* j = (or_job*)arg;
+    or_group_info gi;
+    for (int64_t g = j->lo; g < j->hi; ++g) {
+        or_encode_group(j->t, j->x + g * OR_G, j->blocks + g * OR_BLOCK_BYTES, &gi);
+        j->st.n_groups += 1;
+        j->st.n_nonfinite += (uint64_t)gi.nonfinite;
+        if (gi.zero) { j->st.n_zero += 1; continue; }
+        if (gi.clipped) {
+            j->st.n_clipped += 1;
+            j->st.payload_bits += OR_PAYLOAD_BITS;
+        } else {
+            j->st.payload_bits += (uint64_t)gi.L;
+            if (gi.n_rec > 0) j->st.n_padded += 1;
+            j->st.n_records += (uint64_t)gi.n_rec;
+        }
+        if (j->with_mse) {
+            int pbest = 0;
+            double ebest = INFINITY;
+            for (int p = 0; p < OR_NPAT; ++p) {
+                double e = pattern_mse(j->t, p, gi.u, gi.m);
+                if (e < ebest) { ebest = e; pbest = p; }
+            }
+            j->st.mse_full += ebest;
+            j->st.mse_minmax += pattern_mse(j->t, gi.p, gi.u, gi.m);
+            if (pbest != gi.p) j->st.n_mse_differs += 1;
+        }
+    }
+    return NULL;
+}
+
+static void* decode_worker(void* arg)
+{
+    or_job* j = (or_job*)arg;
+    for (int64_t g = j->lo; g < j->hi; ++g)
+        or_decode_block(j->t, j->blocks + g * OR_BLOCK_BYTES, j->y + g * OR_G);
+    return NULL;
+}
+
+static void run_jobs(void* (*fn)(void*), or_job* base, int64_t n, int nthreads, or_stats* out)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    or_job jobs[256];
+    pthread_t th[256];
+    for (int k = 0; k < nthreads; ++k) {
+        jobs[k] = *base;
+        memset(&jobs[k].st, 0, sizeof jobs[k].st);
+        jobs[k].lo = n * k / nthreads;
+        jobs[k].hi = n * (k + 1) / nthreads;
+    }
+    if (nthreads == 1) fn(&jobs[0]);
+    else {
+        for (int k = 0; k < nthreads; ++k) pthread_create(&th[k], NULL, fn, &jobs[k]);
+        for (int k = 0; k < nthreads; ++k) pthread_join(th[k], NULL);
+    }
+    if (out) {
+        memset(out, 0, sizeof *out);
+        for (int k = 0; k < nthreads; ++k) {
+            out->n_groups += jobs[k].st.n_groups;
+            out->n_zero += jobs[k].st.n_zero;
+            out->n_clipped += jobs[k].st.n_clipped;
+            out->n_padded += jobs[k].st.n_padded;
+            out->n_records += jobs[k].st.n_records;
+            out->n_nonfinite += jobs[k].st.n_nonfinite;
+            out->payload_bits += jobs[k].st.payload_bits;
+            out->n_mse_differs += jobs[k].st.n_mse_differs;
+            out->mse_minmax += jobs[k].st.mse_minmax;
+            out->mse_full += jobs[k].st.mse_full;
+        }
+    }
+}
+
+/* x: n_groups * 128 bf16, contiguous; blocks: n_groups * 64 bytes. */
+void or_encode(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
+               or_stats* stats, int with_mse, int nthreads)
+{
+    or_job base;
+    memset(&base, 0, sizeof base);
+    base.t = t;
+    base.x = x;
+    base.blocks = blocks;
+    base.with_mse = with_mse;
+    run_jobs(encode_worker, &base, n_groups, nthreads, stats);
+}
+
+void or_decode(const or_tables* t, const uint8_t* blocks, int64_t n_blocks, uint16_t* y,
+               int nthreads)
+{
+    or_job base;
+    memset(&base, 0, sizeof base);
+    base.t = t;
+    base.blocks = (uint8_t*)blocks;
+    base.y = y;
+    run_jobs(decode_worker, &base, n_blocks, nthreads, NULL);
+}
+
+/* y[b][r] = sum_k W~[r][k] * x[b][k] in fp64, W~ the decoded blocks of a row-major
+ * rows x cols matrix (cols % 128 == 0), x bf16 [batch][cols].  yabs gets
+ * sum_k |W~[r][k] * x[b][k]| (the scale of the tolerance). */
+void or_gemv(const or_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
+             const uint16_t* x, int batch, double* y, double* yabs)
+{
+    int64_t gpr = cols / OR_G;
+    uint16_t w[OR_G];
+    for (int b = 0; b < batch; ++b)
+        for (int64_t r = 0; r < rows; ++r) {
+            y[(int64_t)b * rows + r] = 0.0;
+            yabs[(int64_t)b * rows + r] = 0.0;
+        }
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < gpr; ++g) {
+            or_decode_block(t, blocks + (r * gpr + g) * OR_BLOCK_BYTES, w);
+            for (int b = 0; b < batch; ++b) {
+                double acc = 0.0, aab = 0.0;
+                for (int i = 0; i < OR_G; ++i) {
+                    double prod = (double)or_bf16_to_f32(w[i]) *
+                                  (double)or_bf16_to_f32(x[(int64_t)b * cols + g * OR_G + i]);
+                    acc += prod;
+                    aab += fabs(prod);
+                }
+                y[(int64_t)b * rows + r] += acc;
+                yabs[(int64_t)b * rows + r] += aab;
+            }
+        }
+}
+
+int or_sizeof_tables(void) { return (int)sizeof(or_tables); }
+int or_sizeof_group_info(void) { return (int)sizeof(or_group_info); }
+int or_sizeof_stats(void) { return (int)sizeof(or_stats); }
