@@ -1,0 +1,541 @@
+#!/usr/bin/env python
+"""Throughput of the Ecco block codec on one or more B200s (one process per GPU).
+
+Default workload (`--workload kv`): one Llama-3-8B-shaped layer of KV cache,
+K and V each [8, 8, 4096, 128] bf16.  A step encodes the last 64 tokens of K
+and V (8,192 groups, written into the compressed cache) and decodes the whole
+compressed cache back to bf16 (524,288 blocks).  Other workloads:
+`c1` (256 x 1024 matrix, encode + decode), `mlp` (14336 x 4096 weight: encode,
+decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights,
+encode and decode of the whole set), `longctx` (32 layers x K,V x
+[1, 8, 131072, 128]: full streaming decode plus a one-token append per layer).
+
+Prints ONE JSON line (rank 0).  `value` is whole-job bf16 GB/s: bf16 bytes the
+step decodes plus bf16 bytes it encodes, over all ranks, per second of device
+time (CUDA events on the launching stream, max over ranks).  L2 is flushed
+between timed steps by writing a 256 MiB buffer outside the step's events.
+`--impl reference` times the CPU oracle on a bounded sample of the same step.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decoded GB/s (bf16 out) & encode GB/s, % of HBM roofline, bit-exact vs oracle"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ecco", choices=["ecco", "reference"])
+    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    """Samples nvidia-smi every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.f.read())) if len(r) >= 9]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads
+class Workload:
+    name = ""
+    desc = ""
+    launches_per_step = 0
+
+    def bytes_decoded(self) -> int:      # bf16 bytes written by decode per step
+        return 0
+
+    def bytes_encoded(self) -> int:      # bf16 bytes read by encode per step
+        return 0
+
+
+def _events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+class KVWorkload(Workload):
+    """One layer of KV cache: encode 64 new tokens, decode the whole cache."""
+    name = "kv"
+    B, H, S, D, T = 8, 8, 4096, 128, 64
+
+    def __init__(self, dev, seed_offset=0):
+        import torch
+        import workloads as W
+        import entropy_coded_kv_b200 as ecco
+        from entropy_coded_kv_b200.calib import learn_tables
+        self.torch, self.ecco, self.dev = torch, ecco, dev
+        self.desc = ("Llama-3-8B-shaped one-layer KV cache, K and V each [8, 8, 4096, 128] bf16: "
+                     "encode the last 64 tokens (8,192 groups) + decode the full cache (524,288 blocks)")
+        K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
+        Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
+        self.tables = [ecco.Tables(learn_tables(Kc, seed=0), dev), ecco.Tables(learn_tables(Vc, seed=0), dev)]
+        self.rows = self.B * self.H
+        self.n = self.rows * self.S
+        self.caches = [K, V]
+        self.blocks = [ecco.encode(K, self.tables[0]), ecco.encode(V, self.tables[1])]
+        self.new = [K.view(self.rows, self.S, self.D)[:, self.S - self.T:].contiguous(),
+                    V.view(self.rows, self.S, self.D)[:, self.S - self.T:].contiguous()]
+        self.out = [torch.empty((self.n, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.append = ecco.kv_append_desc(self.rows, self.T, self.S, self.S - self.T)
+        self.launches_per_step = 4
+        self.dec_ms = []
+
+    def bytes_decoded(self):
+        return 2 * self.n * 256
+
+    def bytes_encoded(self):
+        return 2 * self.rows * self.T * 256
+
+    def step(self, record=False):
+        e = self.ecco
+        for i in range(2):
+            e.encode(self.new[i], self.tables[i], out=self.blocks[i], desc=self.append)
+        for i in range(2):
+            if record:
+                a, b = _events(self.torch)
+                a.record()
+            e.decode(self.blocks[i], self.tables[i], out=self.out[i])
+            if record:
+                b.record()
+                self.dec_ms.append((a, b))
+
+    def dominant(self):
+        """(kernel name, algorithmic bytes per launch, launch ms list)."""
+        self.torch.cuda.synchronize()
+        ms = [a.elapsed_time(b) for a, b in self.dec_ms]
+        return "decode_kernel", self.n * (64 + 256), ms
+
+    # ---- end to end through the public API with host buffers
+    def e2e_setup(self):
+        torch = self.torch
+        self.h_new = [t.cpu().pin_memory() for t in self.new]
+        self.h_blocks = [b.cpu().pin_memory() for b in self.blocks]
+        self.h_out = [torch.empty((self.n, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        self.d_new = [torch.empty_like(t) for t in self.new]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_new + self.h_blocks)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self):
+        e = self.ecco
+        for i in range(2):
+            self.d_new[i].copy_(self.h_new[i], non_blocking=True)
+            self.blocks[i].copy_(self.h_blocks[i], non_blocking=True)
+            e.encode(self.d_new[i], self.tables[i], out=self.blocks[i], desc=self.append)
+            e.decode(self.blocks[i], self.tables[i], out=self.out[i])
+            self.h_out[i].copy_(self.out[i], non_blocking=True)
+
+    # ---- CPU oracle on a bounded sample of the same step
+    def cpu_sample(self, frac):
+        import numpy as np
+        import workloads as W
+        n_dec = max(64, int(self.n * frac))
+        n_enc = max(8, int(self.rows * self.T * frac))
+        xs = [W.bf16_bits(self.new[i].view(-1, 128)[:n_enc]) for i in range(2)]
+        bl = [self.blocks[i][:n_dec].cpu().numpy() for i in range(2)]
+        blobs = [t.blob for t in self.tables]
+        return {"enc": [(blobs[i], xs[i]) for i in range(2)], "dec": [(blobs[i], bl[i]) for i in range(2)],
+                "bytes": 2 * n_dec * 256 + 2 * n_enc * 256,
+                "what": f"encode {2 * n_enc} groups + decode {2 * n_dec} blocks (1/{round(1 / frac)} of a step)"}
+
+
+class C1Workload(Workload):
+    name = "c1"
+
+    def __init__(self, dev, seed_offset=0):
+        import torch
+        import workloads as W
+        import entropy_coded_kv_b200 as ecco
+        from entropy_coded_kv_b200.calib import learn_tables
+        self.torch, self.ecco, self.dev = torch, ecco, dev
+        self.desc = "256 x 1024 bf16 matrix, N(0, 0.02^2) + 0.1% +-20 sigma outliers: encode + decode"
+        self.x = W.c1_matrix(device=dev, seed=0 + seed_offset)
+        self.tables = ecco.Tables(learn_tables(W.c1_matrix(seed=0 + seed_offset)), dev)
+        self.blocks = ecco.encode(self.x, self.tables)
+        self.out = torch.empty((2048, 128), dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = 2
+        self.dec_ms = []
+
+    def bytes_decoded(self):
+        return 2048 * 256
+
+    def bytes_encoded(self):
+        return 2048 * 256
+
+    def step(self, record=False):
+        self.ecco.encode(self.x, self.tables, out=self.blocks)
+        if record:
+            a, b = _events(self.torch)
+            a.record()
+        self.ecco.decode(self.blocks, self.tables, out=self.out)
+        if record:
+            b.record()
+            self.dec_ms.append((a, b))
+
+    def dominant(self):
+        self.torch.cuda.synchronize()
+        return "decode_kernel", 2048 * 320, [a.elapsed_time(b) for a, b in self.dec_ms]
+
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hy = self.torch.empty_like(self.out, device="cpu").pin_memory()
+        self.dx = self.torch.empty_like(self.x)
+        self.h2d, self.d2h = self.hx.numel() * 2, self.hy.numel() * 2
+
+    def e2e_step(self):
+        self.dx.copy_(self.hx, non_blocking=True)
+        self.ecco.encode(self.dx, self.tables, out=self.blocks)
+        self.ecco.decode(self.blocks, self.tables, out=self.out)
+        self.hy.copy_(self.out, non_blocking=True)
+
+    def cpu_sample(self, frac):
+        import workloads as W
+        xb = W.bf16_bits(self.x)
+        return {"enc": [(self.tables.blob, xb)], "dec": [(self.tables.blob, self.blocks.cpu().numpy())],
+                "bytes": 2 * 2048 * 256, "what": "the whole step (encode 2048 groups + decode 2048 blocks)"}
+
+
+class MLPWorkload(Workload):
+    name = "mlp"
+
+    def __init__(self, dev, seed_offset=0):
+        import torch
+        import workloads as W
+        import entropy_coded_kv_b200 as ecco
+        from entropy_coded_kv_b200.calib import learn_tables
+        self.torch, self.ecco, self.dev = torch, ecco, dev
+        self.desc = ("14336 x 4096 bf16 weight, Student-t(5) x 0.02: encode, decode, fused decode+GEMV "
+                     "at batch 1 and batch 16")
+        self.w = W.c3_weight(device=dev, seed=3 + seed_offset)
+        self.rows, self.cols = self.w.shape
+        self.n = self.rows * self.cols // 128
+        self.tables = ecco.Tables(learn_tables(self.w, seed=0), dev)
+        self.blocks = ecco.encode(self.w, self.tables)
+        self.out = torch.empty((self.n, 128), dtype=torch.bfloat16, device=dev)
+        self.x1 = W.activations(self.cols, 1, device=dev)
+        self.x16 = W.activations(self.cols, 16, device=dev)
+        self.y1 = torch.empty((1, self.rows), dtype=torch.float32, device=dev)
+        self.y16 = torch.empty((16, self.rows), dtype=torch.float32, device=dev)
+        self.launches_per_step = 4  # encode, decode, gemv b1, gemv b16 (+2 memsets)
+        self.ev = {"encode": [], "decode": [], "gemv1": [], "gemv16": []}
+
+    def bytes_decoded(self):
+        return self.n * 256
+
+    def bytes_encoded(self):
+        return self.n * 256
+
+    def _t(self, key, fn, record):
+        if record:
+            a, b = _events(self.torch)
+            a.record()
+        fn()
+        if record:
+            b.record()
+            self.ev[key].append((a, b))
+
+    def step(self, record=False):
+        e = self.ecco
+        self._t("encode", lambda: e.encode(self.w, self.tables, out=self.blocks), record)
+        self._t("decode", lambda: e.decode(self.blocks, self.tables, out=self.out), record)
+        self._t("gemv1", lambda: e.decode_gemv(self.blocks, self.tables, self.rows, self.cols, self.x1, out=self.y1), record)
+        self._t("gemv16", lambda: e.decode_gemv(self.blocks, self.tables, self.rows, self.cols, self.x16, out=self.y16), record)
+
+    def dominant(self):
+        self.torch.cuda.synchronize()
+        return "decode_kernel", self.n * 320, [a.elapsed_time(b) for a, b in self.ev["decode"]]
+
+    def per_op(self):
+        self.torch.cuda.synchronize()
+        out = {}
+        byts = {"encode": self.n * 320, "decode": self.n * 320,
+                "gemv1": self.n * 64 + self.cols * 2 + self.rows * 4,
+                "gemv16": self.n * 64 + 16 * self.cols * 2 + 16 * self.rows * 4}
+        for k, evs in self.ev.items():
+            ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+            out[k] = {"ms": ms, "algorithmic_bytes": byts[k], "GB_s": byts[k] / ms / 1e6}
+        return out
+
+    def e2e_setup(self):
+        self.hw = self.w.cpu().pin_memory()
+        self.hx = self.x1.cpu().pin_memory()
+        self.hy = self.torch.empty((self.n, 128), dtype=self.torch.bfloat16).pin_memory()
+        self.hy1 = self.torch.empty((1, self.rows), dtype=self.torch.float32).pin_memory()
+        self.dw = self.torch.empty_like(self.w)
+        self.h2d = self.hw.numel() * 2 + self.hx.numel() * 2
+        self.d2h = self.hy.numel() * 2 + self.hy1.numel() * 4
+
+    def e2e_step(self):
+        e = self.ecco
+        self.dw.copy_(self.hw, non_blocking=True)
+        self.x1.copy_(self.hx, non_blocking=True)
+        e.encode(self.dw, self.tables, out=self.blocks)
+        e.decode(self.blocks, self.tables, out=self.out)
+        e.decode_gemv(self.blocks, self.tables, self.rows, self.cols, self.x1, out=self.y1)
+        e.decode_gemv(self.blocks, self.tables, self.rows, self.cols, self.x16, out=self.y16)
+        self.hy.copy_(self.out, non_blocking=True)
+        self.hy1.copy_(self.y1, non_blocking=True)
+
+    def cpu_sample(self, frac):
+        import workloads as W
+        n = max(64, int(self.n * frac))
+        xb = W.bf16_bits(self.w.view(-1, 128)[:n])
+        return {"enc": [(self.tables.blob, xb)], "dec": [(self.tables.blob, self.blocks[:n].cpu().numpy())],
+                "bytes": 2 * n * 256, "what": f"encode {n} groups + decode {n} blocks (1/{round(1 / frac)} of a step, GEMV not sampled)"}
+
+
+WORKLOADS = {"kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(sample, nthreads):
+    import oracle
+    t0 = time.perf_counter()
+    for blob, xb in sample["enc"]:
+        oracle.encode(blob, xb, nthreads=nthreads)
+    for blob, bl in sample["dec"]:
+        oracle.decode(blob, bl, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, target_s):
+    """The oracle as it stands, on a bounded sample sized for ~target_s seconds."""
+    cores = os.cpu_count() or 1
+    frac = 1.0 / 1024
+    sample = wl.cpu_sample(frac)
+    dt = time_oracle(sample, cores)
+    if dt < target_s / 4 and wl.name != "c1":
+        frac = min(1.0, frac * max(1.0, target_s / max(dt, 1e-3)))
+        sample = wl.cpu_sample(frac)
+        dt = time_oracle(sample, cores)
+    return {"value": sample["bytes"] / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": sample["what"], "seconds": dt}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse_args()
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl" if args.impl == "ecco" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, world)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    from entropy_coded_kv_b200.build import build
+    if rank == 0 or world == 1:
+        build()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = WORKLOADS[args.workload](dev, seed_offset=0)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    for _ in range(max(3, args.warmup)):
+        wl.step()
+        flush.fill_(1.0)
+    torch.cuda.synchronize()
+
+    clk = Clocks(local)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    for i in range(args.steps):
+        starts[i].record()
+        wl.step(record=True)
+        ends[i].record()
+        flush.fill_(1.0)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.stop()
+    ms_total = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    units = (wl.bytes_decoded() + wl.bytes_encoded()) * world
+    value = units / (ms_step * 1e-3) / 1e9
+
+    kname, kbytes, kms = wl.dominant()
+    hbm, src = peaks()
+    k_avg = statistics.mean(kms)
+    achieved = kbytes / (k_avg * 1e-3) / 1e9
+    roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic_for(wl.name, kname),
+            "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
+            "algorithmic_bytes_per_launch": kbytes, "launch_ms": round(k_avg, 5)}
+
+    e2e = None
+    if not args.no_e2e:
+        wl.e2e_setup()
+        for _ in range(2):
+            wl.e2e_step()
+        torch.cuda.synchronize()
+        ks = max(3, min(args.steps, 10))
+        a, b = _events(torch)
+        a.record()
+        for _ in range(ks):
+            wl.e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(b) / ks
+        et = torch.tensor([ems], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        ems = float(et.item())
+        e2e = {"value": round(units / (ems * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ems, 4),
+               "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
+               "api": "entropy_coded_kv_b200.encode/decode (C ABI) with pinned host buffers"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    ops = wl.per_op() if hasattr(wl, "per_op") else None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.desc, "l2": "flushed between steps (256 MiB write outside the step events)",
+                   "decoded_bf16_bytes_per_step": wl.bytes_decoded(),
+                   "encoded_bf16_bytes_per_step": wl.bytes_encoded(),
+                   "parallelism": f"replicas x{world} (independent blocks, no collective)"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": wl.launches_per_step * args.steps,
+    }
+    if ops:
+        line["ops"] = ops
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def traffic_for(workload, kernel):
+    """DRAM bytes per launch from the committed ncu summary, if one matches."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return d.get(f"{workload}:{kernel}")
+
+
+def run_reference(args, world):
+    """The CPU oracle as the reference arm: each step is a bounded sample of the
+    workload, timed with the wall clock on the host cores."""
+    import torch
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
+    if dev is None:
+        print(json.dumps({"impl": "reference", "unavailable": "workload inputs are generated on a CUDA device"}))
+        return
+    wl = WORKLOADS[args.workload](dev)
+    cores = os.cpu_count() or 1
+    frac = 1.0 / 256 if args.workload != "c1" else 1.0
+    sample = wl.cpu_sample(frac)
+    for _ in range(max(1, min(args.warmup, 2))):
+        time_oracle(sample, cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle(sample, cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    v = sample["bytes"] / dt / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.desc, "sample": sample["what"]},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample["what"]},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+"""Ecco 512-bit block codec for LLM tensors on B200 (sm_100a).
+
+Thin PyTorch binding over libecco_b200.so (include/ecco.h): it only turns
+tensors into device pointers and the current CUDA stream into a handle.  Every
+step of encode, decode and decode+GEMV runs in the library's kernels; there is
+no CPU or eager-PyTorch fallback.
+
+Method: "Ecco: Improving Memory Bandwidth and Capacity for LLMs via
+Entropy-aware Cache Compression" (arXiv 2505.06901), review page sections
+"What carries the argument" and "Core claim".
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import EccoError, Desc, Segment, STATS_FIELDS
+
+GROUP = 128
+BLOCK_BYTES = 64
+
+__all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
+           "new_stats", "read_stats", "flat_desc", "kv_append_desc", "EccoError", "Desc"]
+
+
+class Tables:
+    """Device-resident tables of one tensor, built from a table blob (bytes)."""
+
+    def __init__(self, blob: bytes, device=None):
+        lib = _lib.load()
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        if dev.type != "cuda":
+            raise ValueError("tables live on a CUDA device")
+        self.device = dev
+        buf = ctypes.create_string_buffer(bytes(blob), len(blob))
+        h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _lib.check(lib.ecco_tables_create(buf, len(blob), ctypes.byref(h)), "ecco_tables_create")
+        self._h = h
+        self.blob = bytes(blob)
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise ValueError("tables destroyed")
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None:
+            with torch.cuda.device(self.device):
+                _lib.load().ecco_tables_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _stream(dev) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def flat_desc(n_groups: int) -> Desc:
+    return Desc(1, int(n_groups), int(n_groups), int(n_groups), 0, 0)
+
+
+def kv_append_desc(rows: int, new_tokens: int, total_tokens: int, start: int) -> Desc:
+    """Encode [rows, new_tokens] groups from a contiguous tensor into token
+    positions start..start+new_tokens of a [rows, total_tokens] block cache."""
+    return Desc(int(rows), int(new_tokens), int(new_tokens), int(total_tokens), 0, int(start))
+
+
+def _check_tensor(t: torch.Tensor, dtype, name: str, device):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise TypeError(f"{name} must be a {dtype} tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, tables on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def new_stats(device) -> torch.Tensor:
+    """A zeroed device buffer for ecco_stats (8 x u64)."""
+    return torch.zeros(len(STATS_FIELDS), dtype=torch.int64, device=device)
+
+
+def read_stats(stats: torch.Tensor) -> dict:
+    v = stats.cpu().tolist()
+    return {k: int(x) for k, x in zip(STATS_FIELDS, v)}
+
+
+def encode(x: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
+           stats: torch.Tensor | None = None, desc: Desc | None = None) -> torch.Tensor:
+    """bf16 groups of 128 -> uint8 blocks [n_groups, 64].  With `desc`, `x` and
+    `out` are the full source / destination buffers the descriptor indexes."""
+    _check_tensor(x, torch.bfloat16, "x", tables.device)
+    if desc is None:
+        if x.numel() % GROUP:
+            raise ValueError("x.numel() must be a multiple of 128")
+        desc = flat_desc(x.numel() // GROUP)
+    if out is None:
+        if desc.rows * desc.groups_per_row != x.numel() // GROUP or desc.dst_offset:
+            raise ValueError("pass `out` when the descriptor does not map x one-to-one")
+        out = torch.empty((x.numel() // GROUP, BLOCK_BYTES), dtype=torch.uint8, device=x.device)
+    _check_tensor(out, torch.uint8, "out", tables.device)
+    _bounds(desc, x.numel() // GROUP, out.numel() // BLOCK_BYTES)
+    sp = ctypes.c_void_p(stats.data_ptr()) if stats is not None else None
+    rc = _lib.load().ecco_select_encode(tables.handle, ctypes.c_void_p(x.data_ptr()), desc,
+                                        ctypes.c_void_p(out.data_ptr()), sp, _stream(x.device))
+    _lib.check(rc, "ecco_select_encode")
+    return out
+
+
+def decode(blocks: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
+           desc: Desc | None = None) -> torch.Tensor:
+    """uint8 blocks [n, 64] -> bf16 [n, 128]."""
+    _check_tensor(blocks, torch.uint8, "blocks", tables.device)
+    n_blocks = blocks.numel() // BLOCK_BYTES
+    if desc is None:
+        desc = flat_desc(n_blocks)
+    if out is None:
+        out = torch.empty((desc.rows * desc.groups_per_row, GROUP), dtype=torch.bfloat16, device=blocks.device)
+    _check_tensor(out, torch.bfloat16, "out", tables.device)
+    _bounds(desc, n_blocks, out.numel() // GROUP)
+    rc = _lib.load().ecco_decode(tables.handle, ctypes.c_void_p(blocks.data_ptr()), desc,
+                                 ctypes.c_void_p(out.data_ptr()), _stream(blocks.device))
+    _lib.check(rc, "ecco_decode")
+    return out
+
+
+def decode_gemv(blocks: torch.Tensor, tables: Tables, rows: int, cols: int, x: torch.Tensor,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """y[b, r] = sum_k W~[r, k] x[b, k] (fp32), W~ the decoded rows x cols matrix."""
+    _check_tensor(blocks, torch.uint8, "blocks", tables.device)
+    _check_tensor(x, torch.bfloat16, "x", tables.device)
+    if x.dim() == 1:
+        x = x.view(1, -1)
+    batch = x.shape[0]
+    if x.shape[1] != cols or blocks.numel() != rows * (cols // GROUP) * BLOCK_BYTES:
+        raise ValueError("shape mismatch")
+    if out is None:
+        out = torch.empty((batch, rows), dtype=torch.float32, device=x.device)
+    _check_tensor(out, torch.float32, "out", tables.device)
+    rc = _lib.load().ecco_decode_gemv(tables.handle, ctypes.c_void_p(blocks.data_ptr()), rows, cols,
+                                      ctypes.c_void_p(x.data_ptr()), batch,
+                                      ctypes.c_void_p(out.data_ptr()), _stream(x.device))
+    _lib.check(rc, "ecco_decode_gemv")
+    return out
+
+
+@dataclass
+class Seg:
+    tables: Tables
+    src: torch.Tensor
+    dst: torch.Tensor
+    desc: Desc | None = None
+
+
+def _segments(segs, src_dtype, dst_dtype, src_unit, dst_unit):
+    arr = (Segment * max(1, len(segs)))()
+    for i, s in enumerate(segs):
+        _check_tensor(s.src, src_dtype, "src", s.tables.device)
+        _check_tensor(s.dst, dst_dtype, "dst", s.tables.device)
+        d = s.desc or flat_desc(s.src.numel() // src_unit)
+        _bounds(d, s.src.numel() // src_unit, s.dst.numel() // dst_unit)
+        arr[i] = Segment(s.tables.handle, s.src.data_ptr(), s.dst.data_ptr(), d)
+    return arr
+
+
+def decode_multi(segs: list[Seg]) -> None:
+    if not segs:
+        return
+    arr = _segments(segs, torch.uint8, torch.bfloat16, BLOCK_BYTES, GROUP)
+    rc = _lib.load().ecco_decode_multi(arr, len(segs), _stream(segs[0].tables.device))
+    _lib.check(rc, "ecco_decode_multi")
+
+
+def encode_multi(segs: list[Seg], stats: torch.Tensor | None = None) -> None:
+    if not segs:
+        return
+    arr = _segments(segs, torch.bfloat16, torch.uint8, GROUP, BLOCK_BYTES)
+    sp = ctypes.c_void_p(stats.data_ptr()) if stats is not None else None
+    rc = _lib.load().ecco_encode_multi(arr, len(segs), sp, _stream(segs[0].tables.device))
+    _lib.check(rc, "ecco_encode_multi")
+
+
+def _bounds(d: Desc, n_src: int, n_dst: int) -> None:
+    """Host-side check that the descriptor stays inside both buffers."""
+    if d.rows == 0 or d.groups_per_row == 0:
+        return
+    last_src = d.src_offset + (d.rows - 1) * d.src_row_stride + d.groups_per_row
+    last_dst = d.dst_offset + (d.rows - 1) * d.dst_row_stride + d.groups_per_row
+    if min(d.rows, d.groups_per_row, d.src_row_stride, d.dst_row_stride, d.src_offset, d.dst_offset) < 0:
+        raise ValueError("negative descriptor field")
+    if last_src > n_src or last_dst > n_dst:
+        raise ValueError(f"descriptor exceeds buffers (src {last_src}>{n_src} or dst {last_dst}>{n_dst})")

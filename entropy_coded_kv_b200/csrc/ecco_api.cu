@@ -1,0 +1,175 @@
+// C ABI entry points: argument validation, device checks, dispatch to the
+// kernel launchers.  Nothing here allocates device memory.
+#include <cstdint>
+
+#include "ecco_internal.cuh"
+
+namespace ecco {
+
+int device_sm_count()
+{
+    static int cached_dev = -1;
+    static int cached_sms = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != cached_dev) {
+        int sms = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cached_sms = sms > 0 ? sms : 1;
+        cached_dev = dev;
+    }
+    return cached_sms;
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_tables(const ecco_tables* t)
+{
+    if (!t || !t->d) return ECCO_ERR_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ECCO_ERR_CUDA;
+    if (dev != t->device) return ECCO_ERR_DEVICE;
+    return ECCO_OK;
+}
+
+int check_desc(const ecco_desc& d)
+{
+    if (d.rows < 0 || d.groups_per_row < 0 || d.src_row_stride < 0 || d.dst_row_stride < 0 ||
+        d.src_offset < 0 || d.dst_offset < 0)
+        return ECCO_ERR_ARG;
+    if (d.rows > 1 && d.dst_row_stride < d.groups_per_row) return ECCO_ERR_ARG;
+    // keep every group index representable: offset + (rows-1)*stride + gpr < 2^40
+    const int64_t lim = (int64_t)1 << 40;
+    if (d.rows > lim || d.groups_per_row > lim) return ECCO_ERR_ARG;
+    if (d.rows > 0 && d.groups_per_row > 0) {
+        if (d.src_row_stride > lim / (d.rows > 1 ? d.rows : 1)) return ECCO_ERR_ARG;
+        if (d.dst_row_stride > lim / (d.rows > 1 ? d.rows : 1)) return ECCO_ERR_ARG;
+        if (d.src_offset > lim || d.dst_offset > lim) return ECCO_ERR_ARG;
+    }
+    return ECCO_OK;
+}
+
+int status(cudaError_t e) { return e == cudaSuccess ? ECCO_OK : ECCO_ERR_CUDA; }
+
+}  // namespace
+}  // namespace ecco
+
+using namespace ecco;
+
+extern "C" int ecco_select_encode(const ecco_tables* t, const uint16_t* x, ecco_desc d,
+                                  uint8_t* blocks, ecco_stats* stats, void* stream)
+{
+    int rc = check_tables(t);
+    if (rc) return rc;
+    if ((rc = check_desc(d))) return rc;
+    if (d.rows == 0 || d.groups_per_row == 0) return ECCO_OK;
+    if (!x || !blocks) return ECCO_ERR_ARG;
+    if (!aligned16(x) || !aligned16(blocks) || (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return ECCO_ERR_ALIGN;
+    return status(launch_encode(t, x, d, blocks, stats, (cudaStream_t)stream));
+}
+
+extern "C" int ecco_decode(const ecco_tables* t, const uint8_t* blocks, ecco_desc d, uint16_t* y,
+                           void* stream)
+{
+    int rc = check_tables(t);
+    if (rc) return rc;
+    if ((rc = check_desc(d))) return rc;
+    if (d.rows == 0 || d.groups_per_row == 0) return ECCO_OK;
+    if (!blocks || !y) return ECCO_ERR_ARG;
+    if (!aligned16(blocks) || !aligned16(y)) return ECCO_ERR_ALIGN;
+    return status(launch_decode(t, blocks, d, y, (cudaStream_t)stream));
+}
+
+extern "C" int ecco_decode_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows,
+                                int64_t cols, const uint16_t* x, int batch, float* y, void* stream)
+{
+    int rc = check_tables(t);
+    if (rc) return rc;
+    if (rows < 0 || cols < 0 || (cols % ECCO_GROUP) != 0 || batch < 1 || batch > 16)
+        return ECCO_ERR_ARG;
+    if (rows > ((int64_t)1 << 34) || cols > ((int64_t)1 << 34)) return ECCO_ERR_ARG;
+    if (rows == 0) return ECCO_OK;
+    if (!y) return ECCO_ERR_ARG;
+    if (cols == 0) return status(cudaMemsetAsync(y, 0, sizeof(float) * (size_t)batch * (size_t)rows,
+                                                 (cudaStream_t)stream));
+    if (!blocks || !x) return ECCO_ERR_ARG;
+    if (!aligned16(blocks) || !aligned16(x) || !aligned16(y)) return ECCO_ERR_ALIGN;
+    return status(launch_gemv(t, blocks, rows, cols, x, batch, y, (cudaStream_t)stream));
+}
+
+extern "C" int ecco_decode_multi(const ecco_segment* segs, int n, void* stream)
+{
+    if (n < 0 || n > ECCO_MAX_SEGMENTS || (n > 0 && !segs)) return ECCO_ERR_ARG;
+    for (int i = 0; i < n; ++i) {
+        int rc = check_tables(segs[i].tables);
+        if (rc) return rc;
+        if ((rc = check_desc(segs[i].desc))) return rc;
+        if (segs[i].desc.rows == 0 || segs[i].desc.groups_per_row == 0) continue;
+        if (!segs[i].src || !segs[i].dst) return ECCO_ERR_ARG;
+        if (!aligned16(segs[i].src) || !aligned16(segs[i].dst)) return ECCO_ERR_ALIGN;
+    }
+    return status(launch_decode_multi(segs, n, (cudaStream_t)stream));
+}
+
+extern "C" int ecco_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats, void* stream)
+{
+    if (n < 0 || n > ECCO_MAX_SEGMENTS || (n > 0 && !segs)) return ECCO_ERR_ARG;
+    if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return ECCO_ERR_ALIGN;
+    for (int i = 0; i < n; ++i) {
+        int rc = check_tables(segs[i].tables);
+        if (rc) return rc;
+        if ((rc = check_desc(segs[i].desc))) return rc;
+        if (segs[i].desc.rows == 0 || segs[i].desc.groups_per_row == 0) continue;
+        if (!segs[i].src || !segs[i].dst) return ECCO_ERR_ARG;
+        if (!aligned16(segs[i].src) || !aligned16(segs[i].dst)) return ECCO_ERR_ALIGN;
+    }
+    return status(launch_encode_multi(segs, n, stats, (cudaStream_t)stream));
+}
+
+extern "C" const char* ecco_strerror(int code)
+{
+    switch (code) {
+        case ECCO_OK: return "ok";
+        case ECCO_ERR_ARG: return "invalid argument";
+        case ECCO_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ECCO_ERR_TABLES: return "invalid table blob";
+        case ECCO_ERR_CUDA: return "CUDA runtime error";
+        case ECCO_ERR_DEVICE: return "current device is not the tables' device";
+        case ECCO_ERR_UNSUPPORTED: return "device is not sm_100";
+        default: return "unknown error";
+    }
+}
+
+extern "C" int ecco_abi_version(void) { return 1; }
+
+namespace ecco {
+
+// Segments run back to back on the stream, one launch each.
+cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s)
+{
+    for (int i = 0; i < n; ++i) {
+        const ecco_desc& d = segs[i].desc;
+        if (d.rows == 0 || d.groups_per_row == 0) continue;
+        cudaError_t e = launch_decode(segs[i].tables, static_cast<const uint8_t*>(segs[i].src), d,
+                                      static_cast<uint16_t*>(segs[i].dst), s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats, cudaStream_t s)
+{
+    for (int i = 0; i < n; ++i) {
+        const ecco_desc& d = segs[i].desc;
+        if (d.rows == 0 || d.groups_per_row == 0) continue;
+        cudaError_t e = launch_encode(segs[i].tables, static_cast<const uint16_t*>(segs[i].src), d,
+                                      static_cast<uint8_t*>(segs[i].dst), stats, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace ecco

@@ -1,0 +1,116 @@
+// Internal declarations of libecco_b200: device-side table layout, kernel
+// launchers and small device helpers shared by the kernels.
+//
+// Format: "Ecco: Improving Memory Bandwidth and Capacity for LLMs via
+// Entropy-aware Cache Compression" (review page: "What carries the argument",
+// Fig. 4 caption, free parameters).  The bit layout is documented in
+// include/ecco.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ecco.h"
+
+namespace ecco {
+
+constexpr int kG = 128;           // values per group
+constexpr int kNPat = 64;         // shared patterns per tensor
+constexpr int kNCent = 15;        // centroids per pattern
+constexpr int kNBook = 4;         // codebooks per pattern
+constexpr int kNSym = 16;         // symbols (15 centroids + scale element)
+constexpr int kLMax = 8;          // longest codeword
+constexpr int kBlockBits = 512;
+constexpr int kHdrBits = 16;
+constexpr int kPayloadBits = 496;
+constexpr int kRecBits = 15;
+constexpr int kMaxRec = 16;
+
+// Device-resident tables derived once from a blob (ecco_tables_create).
+// Every array a kernel stages into shared memory is 16-byte aligned and a
+// multiple of 16 bytes.
+struct DevTables {
+    float S_t;
+    uint32_t pad0[3];
+    float T16[kNPat][16];           // thresholds (C[j]+C[j+1])*0.5; [14], [15] = +inf
+    float Ct[16][kNPat];            // centroid j of pattern p; row 15 = 1.0 (scale element)
+    float2 ends[kNPat];             // (C[p][0], C[p][14])
+    uint32_t lens4[kNPat][16];      // byte h = length of symbol s in codebook h
+    uint32_t code[kNPat][kNBook][16];  // bits 0-7 codeword in stream order, bits 8-11 length
+    uint8_t lut[kNPat * kNBook][256];  // next 8 stream bits -> symbol | length << 4
+};
+
+}  // namespace ecco
+
+struct ecco_tables {
+    int device;
+    ecco::DevTables* d;
+};
+
+namespace ecco {
+
+// ------------------------------------------------------------ launchers
+struct GridWalk {  // 2-D group index walked with a fixed stride
+    int64_t total;
+    int64_t stride_r, stride_g;  // (gridDim*items per CTA) / gpr, % gpr
+};
+
+cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
+                          uint8_t* blocks, ecco_stats* stats, cudaStream_t s);
+cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
+                          uint16_t* y, cudaStream_t s);
+cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
+                        const uint16_t* x, int batch, float* y, cudaStream_t s);
+cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s);
+cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats,
+                                cudaStream_t s);
+
+int device_sm_count();
+
+// ------------------------------------------------------------ device helpers
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f)
+{
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code)
+{
+    __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+    return __half2float(__half(hr));
+}
+
+// Scale codes whose E4M3 value is zero or NaN mark an all-zero block.
+__device__ __forceinline__ bool scale_code_is_null(uint32_t code)
+{
+    uint32_t mag = code & 0x7fu;
+    return mag == 0u || mag == 0x7fu;
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float warp_min_f32(float v)
+{
+    float r;
+    asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ float warp_max_f32(float v)
+{
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+}  // namespace ecco

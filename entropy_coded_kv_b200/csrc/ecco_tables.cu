@@ -1,0 +1,163 @@
+// Table upload: validates a table blob and derives the device-side tables.
+//
+// The blob holds what the review page says is learned offline per tensor
+// ("Ecco: Improving Memory Bandwidth and Capacity ...", "What carries the
+// argument": 64 patterns of 15 sorted centroids, 4 Huffman codebooks per
+// pattern; Fig. 4 caption: the per-tensor FP8 scale factor).  Derived here:
+//   - thresholds between neighbouring centroids (a value goes to the centroid
+//     whose interval holds it; a value equal to a threshold goes to the lower),
+//   - canonical codewords from the code lengths (ordered by length, then
+//     symbol), stored in stream order (first emitted bit in bit 0),
+//   - a 256-entry decode table per codebook indexed by the next 8 stream bits
+//     (every codeword is at most 8 bits long: referee comment 1, Sec. 4.2).
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "ecco_internal.cuh"
+
+namespace {
+
+using namespace ecco;
+
+struct Blob {
+    uint32_t magic, version;
+    float S_t;
+    uint32_t reserved;
+    float C[kNPat][kNCent];
+    uint8_t len[kNPat][kNBook][kNSym];
+};
+static_assert(sizeof(Blob) == ECCO_TABLES_BYTES, "blob layout");
+
+bool blob_valid(const Blob& b)
+{
+    if (b.magic != ECCO_TABLES_MAGIC || b.version != 1u) return false;
+    if (!std::isfinite(b.S_t) || !(b.S_t >= std::ldexp(1.0f, -60)) || !(b.S_t <= std::ldexp(1.0f, 60)))
+        return false;
+    for (int p = 0; p < kNPat; ++p)
+        for (int j = 0; j < kNCent; ++j) {
+            float c = b.C[p][j];
+            if (!std::isfinite(c) || std::fabs(c) > 4.0f) return false;
+            if (j && !(b.C[p][j - 1] < c)) return false;
+        }
+    for (int p = 0; p < kNPat; ++p)
+        for (int h = 0; h < kNBook; ++h) {
+            unsigned space = 0;  // in units of 2^-kLMax
+            for (int s = 0; s < kNSym; ++s) {
+                unsigned l = b.len[p][h][s];
+                if (l < 1 || l > (unsigned)kLMax) return false;
+                space += 1u << (kLMax - l);
+            }
+            if (space != (1u << kLMax)) return false;  // complete code
+        }
+    return true;
+}
+
+uint32_t reverse_bits(uint32_t v, int n)
+{
+    uint32_t r = 0;
+    for (int i = 0; i < n; ++i) r |= ((v >> i) & 1u) << (n - 1 - i);
+    return r;
+}
+
+// Canonical code values from per-length counts, the construction of RFC 1951
+// section 3.2.2: the first code of length l is (first code of length l-1 +
+// number of codes of length l-1) << 1, and codes of one length are handed out
+// in symbol order.
+void canonical(const uint8_t len[kNSym], uint32_t code[kNSym])
+{
+    uint32_t count[kLMax + 1] = {0};
+    for (int s = 0; s < kNSym; ++s) count[len[s]]++;
+    uint32_t next[kLMax + 1] = {0};
+    for (int l = 2; l <= kLMax; ++l) next[l] = (next[l - 1] + count[l - 1]) << 1;
+    for (int s = 0; s < kNSym; ++s) code[s] = next[len[s]]++;
+}
+
+void derive(const Blob& b, DevTables* t)
+{
+    std::memset(t, 0, sizeof *t);
+    t->S_t = b.S_t;
+    const float inf = INFINITY;
+    for (int p = 0; p < kNPat; ++p) {
+        for (int j = 0; j < kNCent - 1; ++j) {
+            float sum = b.C[p][j] + b.C[p][j + 1];  // rounded on its own (no contraction)
+            t->T16[p][j] = sum * 0.5f;
+        }
+        t->T16[p][14] = inf;
+        t->T16[p][15] = inf;
+        for (int j = 0; j < kNCent; ++j) t->Ct[j][p] = b.C[p][j];
+        t->Ct[15][p] = 1.0f;
+        t->ends[p] = make_float2(b.C[p][0], b.C[p][kNCent - 1]);
+        for (int s = 0; s < kNSym; ++s) {
+            uint32_t v = 0;
+            for (int h = 0; h < kNBook; ++h) v |= (uint32_t)b.len[p][h][s] << (8 * h);
+            t->lens4[p][s] = v;
+        }
+        for (int h = 0; h < kNBook; ++h) {
+            uint32_t code[kNSym];
+            canonical(b.len[p][h], code);
+            uint8_t* lut = t->lut[p * kNBook + h];
+            for (int s = 0; s < kNSym; ++s) {
+                int l = b.len[p][h][s];
+                uint32_t rev = reverse_bits(code[s], l);
+                t->code[p][h][s] = rev | ((uint32_t)l << 8);
+                for (uint32_t tail = 0; tail < (1u << (8 - l)); ++tail)
+                    lut[rev | (tail << l)] = (uint8_t)(s | (l << 4));
+            }
+        }
+    }
+}
+
+}  // namespace
+
+extern "C" int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables** out)
+{
+    if (!blob || !out) return ECCO_ERR_ARG;
+    *out = nullptr;
+    if (nbytes != ECCO_TABLES_BYTES) return ECCO_ERR_TABLES;
+    Blob b;
+    std::memcpy(&b, blob, sizeof b);
+    if (!blob_valid(b)) return ECCO_ERR_TABLES;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ECCO_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ECCO_ERR_CUDA;
+    if (prop.major != 10) return ECCO_ERR_UNSUPPORTED;
+
+    DevTables* host = new (std::nothrow) DevTables;
+    if (!host) return ECCO_ERR_ARG;
+    derive(b, host);
+    DevTables* d = nullptr;
+    if (cudaMalloc(&d, sizeof(DevTables)) != cudaSuccess) {
+        delete host;
+        return ECCO_ERR_CUDA;
+    }
+    cudaError_t e = cudaMemcpy(d, host, sizeof(DevTables), cudaMemcpyHostToDevice);
+    delete host;
+    if (e != cudaSuccess) {
+        cudaFree(d);
+        return ECCO_ERR_CUDA;
+    }
+    ecco_tables* t = new (std::nothrow) ecco_tables;
+    if (!t) {
+        cudaFree(d);
+        return ECCO_ERR_ARG;
+    }
+    t->device = dev;
+    t->d = d;
+    *out = t;
+    return ECCO_OK;
+}
+
+extern "C" int ecco_tables_destroy(ecco_tables* t)
+{
+    if (!t) return ECCO_ERR_ARG;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != t->device) cudaSetDevice(t->device);
+    cudaError_t e = cudaFree(t->d);
+    if (cur != t->device) cudaSetDevice(cur);
+    delete t;
+    return e == cudaSuccess ? ECCO_OK : ECCO_ERR_CUDA;
+}

@@ -1,0 +1,164 @@
+/*
+ * ecco.h -- C ABI of libecco_b200.so, a B200 (sm_100a) implementation of the
+ * Ecco 512-bit block codec for LLM weight and KV-cache tensors.
+ *
+ * Method: "Ecco: Improving Memory Bandwidth and Capacity for LLMs via
+ * Entropy-aware Cache Compression" (arXiv 2505.06901; pith.science review page).
+ * Every 128-value bf16 group becomes one self-contained 64-byte block holding a
+ * per-group FP8 scale, a pattern index (one of 64 shared 15-centroid k-means
+ * patterns, chosen by min/max), a codebook choice (the shortest of 4 Huffman
+ * codebooks), the Huffman-coded centroid indices, and padded outliers
+ * (review page: "What carries the argument", "Core claim", Fig. 4 caption,
+ * free-parameter list).
+ *
+ * Block layout (the page gives the fields, not their bit positions; these are
+ * the library's readings):
+ *   stream bit b = bit (b % 8) of byte b / 8 (little-endian 32-bit words);
+ *   bits 0-7   FP8 E4M3 scale code (signed; codes 0x00/0x80/0x7f/0xff decode
+ *              to a block of 128 zeros);
+ *   bits 8-13  pattern index p (0..63);
+ *   bits 14-15 codebook index h (0..3);
+ *   bits 16-   canonical Huffman codewords of the 128 symbols in element order,
+ *              each written most-significant code bit first (lengths 1..8).
+ *              Symbol 15 is the scale element (value = s).  A codeword that
+ *              does not fit below bit 512 is cut there and ends the stream
+ *              ("clip the excess"); elements from it on decode to +0.
+ *   unclipped blocks with L payload bits then carry n = min(16, (496-L)/15)
+ *   outlier records of 15 bits: element index (7 bits) then q (8-bit two's
+ *   complement), decoded as bf16(s * (q / 127)) over the centroid value.
+ * Decoded value of element i: bf16 round-half-even of fp32(s * C[p][sym_i]).
+ *
+ * Conventions for every call:
+ *   - Data pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or retains them.  Table objects are library-owned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous: they validate, enqueue kernels and return.
+ *   - The calling thread's current device must be the device the tables were
+ *     created on.
+ *   - Return value: ECCO_OK or a negative ECCO_ERR_* code.  On an argument
+ *     error nothing is enqueued.  Data-dependent conditions (non-finite input,
+ *     clipping) are never errors; they are counted in ecco_stats.
+ */
+#ifndef ECCO_H
+#define ECCO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ECCO_OK 0
+#define ECCO_ERR_ARG (-1)         /* null/negative/inconsistent argument */
+#define ECCO_ERR_ALIGN (-2)       /* pointer not 16-byte aligned */
+#define ECCO_ERR_TABLES (-3)      /* table blob invalid */
+#define ECCO_ERR_CUDA (-4)        /* CUDA runtime error (launch, copy, device) */
+#define ECCO_ERR_DEVICE (-5)      /* current device is not the tables' device */
+#define ECCO_ERR_UNSUPPORTED (-6) /* device is not sm_100 */
+
+#define ECCO_GROUP 128            /* values per group */
+#define ECCO_BLOCK_BYTES 64       /* bytes per compressed block (512 bits) */
+#define ECCO_NPAT 64              /* shared k-means patterns per tensor */
+#define ECCO_NCENT 15             /* sorted centroids per pattern */
+#define ECCO_NBOOK 4              /* Huffman codebooks per pattern */
+#define ECCO_NSYM 16              /* symbols: 15 centroids + the scale element */
+#define ECCO_LMAX 8               /* longest codeword, bits */
+#define ECCO_TABLES_MAGIC 0x31434345u
+#define ECCO_TABLES_BYTES 7952u
+
+/* Table blob (host memory, little-endian), the per-tensor parameters learned
+ * offline ("64 patterns per tensor", "4 Huffman codebooks per pattern"):
+ *   u32 magic = ECCO_TABLES_MAGIC, u32 version = 1, f32 S_t, u32 reserved,
+ *   f32 C[64][15]      centroids, strictly increasing per pattern, |C| <= 4,
+ *   u8  len[64][4][16] code lengths 1..8, Kraft sum exactly 1 per codebook.
+ * S_t is the per-tensor FP8 scale factor (Fig. 4 caption), normal, in
+ * [2^-60, 2^60]. */
+typedef struct ecco_tables ecco_tables;
+
+/* A 2-D array of groups.  Group (r, g), 0 <= r < rows, 0 <= g < groups_per_row,
+ * is read at source group index  src_offset + r * src_row_stride + g  and
+ * written at destination index   dst_offset + r * dst_row_stride + g.
+ * A group index addresses 128 bf16 values (256 bytes) on the bf16 side and one
+ * 64-byte block on the compressed side.  A flat tensor is rows = 1.  Writing
+ * the last T tokens of a [B, H, S, 128] KV cache from a [B, H, T, 128] tensor:
+ * rows = B*H, groups_per_row = T, src_row_stride = T, dst_row_stride = S,
+ * src_offset = 0, dst_offset = S - T.  All fields >= 0; when rows > 1,
+ * dst_row_stride >= groups_per_row (destination rows may not overlap). */
+typedef struct {
+    int64_t rows;
+    int64_t groups_per_row;
+    int64_t src_row_stride;
+    int64_t dst_row_stride;
+    int64_t src_offset;
+    int64_t dst_offset;
+} ecco_desc;
+
+/* Per-call counters, accumulated (atomically added) into a caller-owned device
+ * struct that the caller zeroes.  n_padded counts unclipped blocks with at
+ * least one outlier record; payload_bits sums min(L, 496) over non-zero blocks
+ * (clip and padding ratios as in the review page's Fig. 10). */
+typedef struct {
+    unsigned long long n_groups;
+    unsigned long long n_zero;
+    unsigned long long n_clipped;
+    unsigned long long n_padded;
+    unsigned long long n_records;
+    unsigned long long n_nonfinite;
+    unsigned long long payload_bits;
+    unsigned long long reserved;
+} ecco_stats;
+
+/* Validates `blob` (nbytes == ECCO_TABLES_BYTES), derives the device-side
+ * tables (thresholds, canonical codes, decode lookup tables) and uploads them
+ * to the current device.  Blocking; not for the hot path.  On success *out
+ * owns device memory until ecco_tables_destroy. */
+int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables** out);
+int ecco_tables_destroy(ecco_tables* tables);
+
+/* Encoder ("Core claim"; "What carries the argument"): for every group of
+ * `x_bf16` described by `desc`, picks the FP8 scale, the pattern by min/max
+ * squared error, the symbols, the shortest codebook, packs and clips the
+ * codewords and pads outliers, and writes one 64-byte block to `blocks`.
+ * `dev_stats` may be NULL.  x_bf16 and blocks must be 16-byte aligned. */
+int ecco_select_encode(const ecco_tables* tables, const uint16_t* x_bf16, ecco_desc desc,
+                       uint8_t* blocks, ecco_stats* dev_stats, void* stream);
+
+/* Decoder (the review page's decompressor, Fig. 8 caption): every block of
+ * `blocks` described by `desc` becomes 128 bf16 values in `y_bf16`.  Any
+ * 64-byte pattern decodes deterministically (malformed blocks included).
+ * blocks and y_bf16 must be 16-byte aligned. */
+int ecco_decode(const ecco_tables* tables, const uint8_t* blocks, ecco_desc desc,
+                uint16_t* y_bf16, void* stream);
+
+/* Fused decode + matrix-vector product ("Normalized memory requests for a
+ * GEMM kernel", review page figure list): y[b][r] = sum_k W~[r][k] x[b][k],
+ * W~ the decoded rows x cols matrix whose blocks are stored row-major
+ * (block (r, g) at index r * cols/128 + g), x_bf16 [batch][cols], y [batch][rows]
+ * fp32.  cols % 128 == 0, 1 <= batch <= 16.  The decoded matrix is never
+ * written to memory.  Accumulation order is unspecified (fp32). */
+int ecco_decode_gemv(const ecco_tables* tables, const uint8_t* blocks, int64_t rows,
+                     int64_t cols, const uint16_t* x_bf16, int batch, float* y, void* stream);
+
+/* Many tensors in one launch: segment i decodes (or encodes) with its own
+ * tables.  At most ECCO_MAX_SEGMENTS per call; arrays are host memory, read
+ * before the call returns. */
+#define ECCO_MAX_SEGMENTS 256
+typedef struct {
+    const ecco_tables* tables;
+    const void* src; /* blocks (decode) / bf16 values (encode) */
+    void* dst;       /* bf16 values (decode) / blocks (encode) */
+    ecco_desc desc;
+} ecco_segment;
+
+int ecco_decode_multi(const ecco_segment* segments, int n_segments, void* stream);
+int ecco_encode_multi(const ecco_segment* segments, int n_segments, ecco_stats* dev_stats,
+                      void* stream);
+
+const char* ecco_strerror(int code);
+int ecco_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ECCO_H */
