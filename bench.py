@@ -19,15 +19,11 @@ between timed steps by writing a 256 MiB buffer outside the step's events.
 from __future__ import annotations
 
 import argparse
-import csv
 import datetime
-import io
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -61,49 +57,66 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks
 class Clocks:
-    """Samples nvidia-smi every 200 ms while the timed region runs."""
+    """Polls NVML (read-only) every millisecond while the timed region runs:
+    SM clock, its maximum, and the active clock-event (throttle) reasons."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.f = None
+    def __init__(self, torch_dev):
+        self.dev = torch_dev
+        self.samples = []
+        self.reasons = set()
+        self.h = None
+        self._stop = None
+        self._th = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
 
     def start(self):
+        import threading
         try:
-            self.f = tempfile.TemporaryFile(mode="w+")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            self.h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report it, do not guess
+            self.h = None
+            self.err = str(e)
+            return
+        self._stop = threading.Event()
+
+        def poll():
+            import pynvml
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    for bit, name in self.REASONS.items():
+                        if r & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                self._stop.wait(0.001)
+
+        self._th = threading.Thread(target=poll, daemon=True)
+        self._th.start()
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.seek(0)
-        rows = [r for r in csv.reader(io.StringIO(self.f.read())) if len(r) >= 9]
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvml unavailable: {getattr(self, 'err', '')}"]}
+        self._stop.set()
+        self._th.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ workloads
@@ -114,6 +127,9 @@ class Workload:
 
     def bytes_decoded(self) -> int:      # bf16 bytes written by decode per step
         return 0
+
+    def cpu_frac(self) -> float:         # fraction of a step the oracle samples (~1 s of host work)
+        return 1.0
 
     def bytes_encoded(self) -> int:      # bf16 bytes read by encode per step
         return 0
@@ -368,17 +384,18 @@ def time_oracle(sample, nthreads):
 
 
 def cpu_baseline(wl, target_s):
-    """The oracle as it stands, on a bounded sample sized for ~target_s seconds."""
+    """The oracle as it stands, on a bounded sample of the step, repeated until
+    about target_s seconds of host work have been timed."""
     cores = os.cpu_count() or 1
-    frac = 1.0 / 1024
+    frac = wl.cpu_frac()
     sample = wl.cpu_sample(frac)
     dt = time_oracle(sample, cores)
-    if dt < target_s / 4 and wl.name != "c1":
-        frac = min(1.0, frac * max(1.0, target_s / max(dt, 1e-3)))
-        sample = wl.cpu_sample(frac)
-        dt = time_oracle(sample, cores)
-    return {"value": sample["bytes"] / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": sample["what"], "seconds": dt}
+    reps, total = 1, dt
+    while total < target_s and reps < 1000:
+        total += time_oracle(sample, cores)
+        reps += 1
+    return {"value": sample["bytes"] * reps / total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{sample['what']}, {reps} repetitions", "seconds": round(total, 2)}
 
 
 # ------------------------------------------------------------------ main
@@ -416,7 +433,7 @@ def main():
         flush.fill_(1.0)
     torch.cuda.synchronize()
 
-    clk = Clocks(local)
+    clk = Clocks(dev)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
@@ -517,8 +534,7 @@ def run_reference(args, world):
         return
     wl = WORKLOADS[args.workload](dev)
     cores = os.cpu_count() or 1
-    frac = 1.0 / 256 if args.workload != "c1" else 1.0
-    sample = wl.cpu_sample(frac)
+    sample = wl.cpu_sample(wl.cpu_frac())
     for _ in range(max(1, min(args.warmup, 2))):
         time_oracle(sample, cores)
     t0 = time.perf_counter()

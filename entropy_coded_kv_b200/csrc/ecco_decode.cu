@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
               q3 = ldg_nc_v4(src + 48);
         const uint32_t code = q0.x & 0xffu;
         const int p = (int)((q0.x >> 8) & 63u);
-        const int cb = (int)((q0.x >> 8) & 255u);  // p * 4 + h
+        const int cb = (int)((q0.x >> 8) & 255u);  // h * 64 + p: the decode table index
         if (scale_code_is_null(code)) {
 #pragma unroll
             for (int k = 0; k < 16; ++k) stg128(dst + 8 * k, 0u, 0u, 0u, 0u);

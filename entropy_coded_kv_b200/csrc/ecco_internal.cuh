@@ -39,7 +39,7 @@ struct DevTables {
     float2 ends[kNPat];             // (C[p][0], C[p][14])
     uint32_t lens4[kNPat][16];      // byte h = length of symbol s in codebook h
     uint32_t code[kNPat][kNBook][16];  // bits 0-7 codeword in stream order, bits 8-11 length
-    uint8_t lut[kNPat * kNBook][256];  // next 8 stream bits -> symbol | length << 4
+    uint8_t lut[kNBook * kNPat][256];  // [h * 64 + p] (= header bits 8-15): next 8 stream bits -> symbol | length << 4
 };
 
 }  // namespace ecco

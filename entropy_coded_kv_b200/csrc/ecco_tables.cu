@@ -96,7 +96,7 @@ void derive(const Blob& b, DevTables* t)
         for (int h = 0; h < kNBook; ++h) {
             uint32_t code[kNSym];
             canonical(b.len[p][h], code);
-            uint8_t* lut = t->lut[p * kNBook + h];
+            uint8_t* lut = t->lut[h * kNPat + p];
             for (int s = 0; s < kNSym; ++s) {
                 int l = b.len[p][h][s];
                 uint32_t rev = reverse_bits(code[s], l);
