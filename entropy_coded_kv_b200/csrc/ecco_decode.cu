@@ -6,35 +6,40 @@
 // offset to beat the serial dependency of one variable-length stream.  A
 // B200 has millions of independent blocks in flight instead, so here every
 // thread walks one block's stream serially and parallelism comes from the
-// blocks: the latency of the serial chain (one shared-memory lookup per
-// symbol) is hidden by 32 resident warps per SM, and no work is spent on
-// offsets that turn out to be wrong.
+// blocks: the serial chain (one shared-memory table lookup per symbol) is
+// hidden by 32 resident warps per SM, and no work is spent on offsets that
+// turn out to be wrong.
 //
-// Per block: parse the header (scale code, pattern, codebook), build the
-// block's 16 output values bf16(s * C[p][j]) in a per-thread slot of shared
-// memory, then for every symbol look up (symbol, length) from the next 8
-// stream bits in the codebook's 256-entry table, emit the value, and stop
-// emitting at the first codeword that would cross bit 512 (clipping).  An
-// unclipped stream is followed by min(16, (496 - L) / 15) outlier records.
-#include "ecco_internal.cuh"
+// Per block: parse the header (scale code, pattern, codebook), form the 16
+// output values bf16(s * C[p][j]) as register byte planes, decode the stream
+// 8 symbols at a time (ecco_block.cuh), write each 16 decoded values with one
+// 32-byte store, then apply the outlier records of an unclipped stream.
+#include "ecco_block.cuh"
 
 namespace ecco {
 namespace {
 
 constexpr int kDecThreads = 1024;
-constexpr int kWordStride = kDecThreads + 2;  // keeps cooperative stores conflict-free
+constexpr int kWordStride = kDecThreads;  // word k of thread t at k * stride + t: conflict-free
 
 constexpr size_t kDecSmemLut = sizeof(((DevTables*)0)->lut);  // 65536
 constexpr size_t kDecSmemCt = sizeof(((DevTables*)0)->Ct);    // 4096
-constexpr size_t kDecSmemVt = 16 * kDecThreads * 4;
 constexpr size_t kDecSmemWords = 16 * kWordStride * 4;
-constexpr size_t kDecSmem = kDecSmemLut + kDecSmemCt + kDecSmemVt + kDecSmemWords;
+constexpr size_t kDecSmem = kDecSmemLut + kDecSmemCt + kDecSmemWords;
 
-__device__ __forceinline__ void stg128(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+// WIDE: 32-byte stores (output 32-byte aligned), else 16-byte stores.
+template <bool WIDE>
+__device__ __forceinline__ void store16(uint16_t* dst, const uint32_t a[4], const uint32_t b[4])
 {
-    *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
+    if (WIDE) {
+        stg256(dst, a, b);
+    } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(a[0], a[1], a[2], a[3]);
+        *reinterpret_cast<uint4*>(dst + 8) = make_uint4(b[0], b[1], b[2], b[3]);
+    }
 }
 
+template <bool WIDE>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const DevTables* __restrict__ tb, const uint8_t* __restrict__ blocks, ecco_desc d,
                   uint16_t* __restrict__ y, GridWalk walk)
@@ -42,8 +47,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kDecSmemLut);
-    uint32_t* s_vt = reinterpret_cast<uint32_t*>(smem + kDecSmemLut + kDecSmemCt);
-    uint32_t* s_w = s_vt + 16 * kDecThreads;
+    uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kDecSmemLut + kDecSmemCt);
     const int tid = threadIdx.x;
     {
         const uint4* a = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
@@ -56,9 +60,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const float S_t = tb->S_t;
     __syncthreads();
 
-    uint32_t* vt = s_vt + tid;  // value j at vt[j * kDecThreads]
-    uint32_t* ws = s_w + tid;   // word k at ws[k * kWordStride]
-
+    uint32_t* ws = s_w + tid;
     const int64_t gpr = d.groups_per_row;
     int64_t item = (int64_t)blockIdx.x * kDecThreads + tid;
     int64_t r = item / gpr, g = item - r * gpr;
@@ -75,79 +77,32 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         uint4 q0 = ldg_nc_v4(src), q1 = ldg_nc_v4(src + 16), q2 = ldg_nc_v4(src + 32),
               q3 = ldg_nc_v4(src + 48);
         const uint32_t code = q0.x & 0xffu;
-        const int p = (int)((q0.x >> 8) & 63u);
-        const int cb = (int)((q0.x >> 8) & 255u);  // h * 64 + p: the decode table index
         if (scale_code_is_null(code)) {
+            const uint32_t z[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int k = 0; k < 16; ++k) stg128(dst + 8 * k, 0u, 0u, 0u, 0u);
+            for (int k = 0; k < 8; ++k) store16<WIDE>(dst + 16 * k, z, z);
             continue;
         }
-        ws[2 * kWordStride] = q0.z;
-        ws[3 * kWordStride] = q0.w;
-        ws[4 * kWordStride] = q1.x;
-        ws[5 * kWordStride] = q1.y;
-        ws[6 * kWordStride] = q1.z;
-        ws[7 * kWordStride] = q1.w;
-        ws[8 * kWordStride] = q2.x;
-        ws[9 * kWordStride] = q2.y;
-        ws[10 * kWordStride] = q2.z;
-        ws[11 * kWordStride] = q2.w;
-        ws[12 * kWordStride] = q3.x;
-        ws[13 * kWordStride] = q3.y;
-        ws[14 * kWordStride] = q3.z;
-        ws[15 * kWordStride] = q3.w;
-
+        stage_words(ws, kWordStride, q0, q1, q2, q3);
+        const int p = (int)((q0.x >> 8) & 63u);
+        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;  // table h * 64 + p
         const float s = __fmul_rn(S_t, e4m3_to_f32(code));
-#pragma unroll
-        for (int j = 0; j < 16; ++j) vt[j * kDecThreads] = f32_to_bf16_bits(__fmul_rn(s, s_Ct[j * kNPat + p]));
+        const ValuePlanes vp = make_planes(s, s_Ct, p);
 
-        const uint8_t* lut = s_lut + cb * 256;
-        uint32_t lo = q0.x, hi = q0.y;
-        int b = kHdrBits;       // bit offset of the window (lo, hi)
-        int widx = 2;           // next word to load
-        int room = kBlockBits - kHdrBits;  // bits left before the block end
-        bool valid = true;
-        uint32_t out[4];
+        Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 #pragma unroll 1
-        for (int c = 0; c < 16; ++c) {  // 16 chunks of 8 symbols
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                if (b >= 32) {
-                    lo = hi;
-                    hi = (widx < 16) ? ws[widx * kWordStride] : 0u;
-                    widx++;
-                    b -= 32;
-                }
-                uint32_t cur = __funnelshift_r(lo, hi, b);
-                int used = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t e = lut[cur & 0xffu];
-                    int len = (int)(e >> 4);
-                    cur >>= len;
-                    used += len;
-                    valid = valid && (used <= room);
-                    uint32_t v = valid ? vt[(e & 15u) * kDecThreads] : 0u;
-                    if (j & 1)
-                        out[half * 2 + (j >> 1)] |= v << 16;
-                    else
-                        out[half * 2 + (j >> 1)] = v;
-                }
-                b += used;
-                room -= used;
-            }
-            stg128(dst + 8 * c, out[0], out[1], out[2], out[3]);
+        for (int c = 0; c < 8; ++c) {  // 8 x 16 symbols, one 32-byte store each
+            uint32_t wa[4], wb[4];
+            chunk_values(st, lut, ws, kWordStride, vp, wa);
+            chunk_values(st, lut, ws, kWordStride, vp, wb);
+            store16<WIDE>(dst + 16 * c, wa, wb);
         }
 
-        if (valid) {  // unclipped: outlier records follow the codewords
-            int L = kPayloadBits - room;
-            int n = min(kMaxRec, room / kRecBits);
-            int at = kHdrBits + L;
+        if (st.room >= 0) {  // unclipped: outlier records follow the codewords
+            const int n = min(kMaxRec, st.room / kRecBits);
+            int at = kBlockBits - st.room;
             for (int k = 0; k < n; ++k, at += kRecBits) {
-                int wi = at >> 5;
-                uint32_t w0 = (wi < 2) ? ((wi == 0) ? q0.x : q0.y) : ws[wi * kWordStride];
-                uint32_t w1 = (wi + 1 < 2) ? q0.y : ((wi + 1 < 16) ? ws[(wi + 1) * kWordStride] : 0u);
-                uint32_t rec = __funnelshift_r(w0, w1, at & 31) & 0x7fffu;
+                uint32_t rec = read_record(ws, kWordStride, at);
                 int i = (int)(rec & 127u);
                 int qv = (int)(int8_t)(uint8_t)(rec >> 7);
                 float o = __fdiv_rn((float)qv, 127.0f);
@@ -165,8 +120,11 @@ cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecc
     static int configured_dev = -1;
     int dev = t->device;
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kDecSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kDecSmem);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
@@ -179,7 +137,10 @@ cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecc
     int64_t stride = (int64_t)grid * kDecThreads;
     walk.stride_r = stride / d.groups_per_row;
     walk.stride_g = stride % d.groups_per_row;
-    decode_kernel<<<grid, kDecThreads, kDecSmem, s>>>(t->d, blocks, d, y, walk);
+    if ((reinterpret_cast<uintptr_t>(y) & 31u) == 0)
+        decode_kernel<true><<<grid, kDecThreads, kDecSmem, s>>>(t->d, blocks, d, y, walk);
+    else
+        decode_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(t->d, blocks, d, y, walk);
     return cudaGetLastError();
 }
 

@@ -12,7 +12,7 @@
 // record replaces the value of its element, so its contribution is corrected
 // by (new - old) * x, with the old symbol kept in shared memory.  Partial row
 // sums of the column ranges are combined with fp32 atomics.
-#include "ecco_internal.cuh"
+#include "ecco_block.cuh"
 
 namespace ecco {
 namespace {
@@ -20,18 +20,17 @@ namespace {
 constexpr int kGvThreads = 512;
 constexpr int kGvWarps = kGvThreads / 32;
 constexpr int kGvColGroups = 4;   // column groups per CTA (x slice of 512 values)
-constexpr int kGvStride = kGvThreads + 2;
+constexpr int kGvStride = kGvThreads;
 
 constexpr size_t kGvLut = 65536;
 constexpr size_t kGvCt = 4096;
-constexpr size_t kGvVt = 16 * kGvThreads * 4;
 constexpr size_t kGvWords = 16 * kGvStride * 4;
 constexpr size_t kGvNib = 16 * kGvThreads * 4;
 
 template <int B>
 constexpr size_t gv_smem()
 {
-    return kGvLut + kGvCt + kGvVt + kGvWords + kGvNib + (size_t)kGvColGroups * kG * B * 4;
+    return kGvLut + kGvCt + kGvWords + kGvNib + (size_t)kGvColGroups * kG * B * 4;
 }
 
 template <int B>
@@ -43,8 +42,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kGvLut);
-    float* s_vt = reinterpret_cast<float*>(smem + kGvLut + kGvCt);
-    uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kGvLut + kGvCt + kGvVt);
+    uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kGvLut + kGvCt);
     uint32_t* s_nib = s_w + 16 * kGvStride;
     float* s_x = reinterpret_cast<float*>(s_nib + 16 * kGvThreads);  // [k][B]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -70,9 +68,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 
     const int64_t row = ((int64_t)blockIdx.x * kGvWarps + warp) * 32 + lane;
     const bool row_ok = row < rows;
-    float* vt = s_vt + tid;
     uint32_t* ws = s_w + tid;
-    uint32_t* nib = s_nib + tid;
+    uint32_t* nibs = s_nib + tid;
     float acc[B];
 #pragma unroll
     for (int bb = 0; bb < B; ++bb) acc[bb] = 0.0f;
@@ -89,86 +86,42 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         }
         const uint32_t code = q0.x & 0xffu;
         const int p = (int)((q0.x >> 8) & 63u);
-        const int cb = (int)((q0.x >> 8) & 255u);
-        const bool live = row_ok && !scale_code_is_null(code);
-        ws[2 * kGvStride] = q0.z;
-        ws[3 * kGvStride] = q0.w;
-        ws[4 * kGvStride] = q1.x;
-        ws[5 * kGvStride] = q1.y;
-        ws[6 * kGvStride] = q1.z;
-        ws[7 * kGvStride] = q1.w;
-        ws[8 * kGvStride] = q2.x;
-        ws[9 * kGvStride] = q2.y;
-        ws[10 * kGvStride] = q2.z;
-        ws[11 * kGvStride] = q2.w;
-        ws[12 * kGvStride] = q3.x;
-        ws[13 * kGvStride] = q3.y;
-        ws[14 * kGvStride] = q3.z;
-        ws[15 * kGvStride] = q3.w;
-        const float s = __fmul_rn(S_t, e4m3_to_f32(code));
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            vt[j * kGvThreads] = live ? bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, s_Ct[j * kNPat + p]))) : 0.0f;
+        // a row past the end or a null scale contributes zeros
+        const float s = (row_ok && !scale_code_is_null(code)) ? __fmul_rn(S_t, e4m3_to_f32(code)) : 0.0f;
+        stage_words(ws, kGvStride, q0, q1, q2, q3);
+        const ValuePlanes vp = make_planes(s, s_Ct, p);
+        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
 
-        const uint8_t* lut = s_lut + cb * 256;
-        uint32_t lo = q0.x, hi = q0.y;
-        int b = kHdrBits, widx = 2, room = kBlockBits - kHdrBits;
-        bool valid = true;
+        Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 #pragma unroll 1
         for (int c = 0; c < 16; ++c) {
-            uint32_t nb = 0;
+            uint32_t w[4];
+            nibs[c * kGvThreads] = chunk_values(st, lut, ws, kGvStride, vp, w);
+            const float* xk = xs + c * 8 * B;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                if (b >= 32) {
-                    lo = hi;
-                    hi = (widx < 16) ? ws[widx * kGvStride] : 0u;
-                    widx++;
-                    b -= 32;
-                }
-                uint32_t cur = __funnelshift_r(lo, hi, b);
-                int used = 0;
+            for (int j = 0; j < 8; ++j) {
+                float v = __uint_as_float((j & 1) ? (w[j >> 1] & 0xffff0000u) : (w[j >> 1] << 16));
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t e = lut[cur & 0xffu];
-                    int len = (int)(e >> 4);
-                    cur >>= len;
-                    used += len;
-                    valid = valid && (used <= room);
-                    uint32_t sym = e & 15u;
-                    nb |= sym << (4 * (half * 4 + j));
-                    float v = valid ? vt[sym * kGvThreads] : 0.0f;
-                    const float* xk = xs + (c * 8 + half * 4 + j) * B;
-#pragma unroll
-                    for (int bb = 0; bb < B; ++bb) acc[bb] = fmaf(v, xk[bb], acc[bb]);
-                }
-                b += used;
-                room -= used;
+                for (int bb = 0; bb < B; ++bb) acc[bb] = fmaf(v, xk[j * B + bb], acc[bb]);
             }
-            nib[c * kGvThreads] = nb;
         }
-        if (live && valid) {
-            int L = kPayloadBits - room;
-            int n = min(kMaxRec, room / kRecBits);
-            int at0 = kHdrBits + L;
-            for (int k = n - 1; k >= 0; --k) {  // last record of an element wins
-                int at = at0 + k * kRecBits;
-                int wi = at >> 5;
-                uint32_t rec = __funnelshift_r(ws[wi * kGvStride], (wi + 1 < 16) ? ws[(wi + 1) * kGvStride] : 0u,
-                                               at & 31) & 0x7fffu;
+        if (s != 0.0f && st.room >= 0) {  // outlier records replace their element's value
+            const int n = min(kMaxRec, st.room / kRecBits);
+            const int at0 = kBlockBits - st.room;
+            for (int k = n - 1; k >= 0; --k) {  // the last record of an element wins
+                uint32_t rec = read_record(ws, kGvStride, at0 + k * kRecBits);
                 int i = (int)(rec & 127u);
                 bool later = false;
-                for (int k2 = k + 1; k2 < n; ++k2) {
-                    int a2 = at0 + k2 * kRecBits;
-                    int w2 = a2 >> 5;
-                    uint32_t r2 = __funnelshift_r(ws[w2 * kGvStride], (w2 + 1 < 16) ? ws[(w2 + 1) * kGvStride] : 0u,
-                                                  a2 & 31);
-                    later = later || ((int)(r2 & 127u) == i);
-                }
+                for (int k2 = k + 1; k2 < n; ++k2)
+                    later = later || ((int)(read_record(ws, kGvStride, at0 + k2 * kRecBits) & 127u) == i);
                 if (later) continue;
                 int qv = (int)(int8_t)(uint8_t)(rec >> 7);
                 float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __fdiv_rn((float)qv, 127.0f))));
-                uint32_t osym = (nib[(i >> 3) * kGvThreads] >> (4 * (i & 7))) & 15u;
-                float ov = vt[osym * kGvThreads];
+                uint32_t osym = (nibs[(i >> 3) * kGvThreads] >> (4 * (i & 7))) & 15u;
+                uint32_t ow = (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);
+                uint32_t oh = (osym < 8) ? ((osym < 4) ? vp.hi[0] : vp.hi[1]) : ((osym < 12) ? vp.hi[2] : vp.hi[3]);
+                uint32_t sh = 8 * (osym & 3);
+                float ov = __uint_as_float((((ow >> sh) & 0xffu) | (((oh >> sh) & 0xffu) << 8)) << 16);
                 float dv = nv - ov;
                 const float* xi = xs + i * B;
 #pragma unroll

@@ -145,6 +145,20 @@ def test_ragged_sizes(n):
     np.testing.assert_array_equal(bits(y).reshape(-1, 128), oracle.decode(blob, want, nthreads=8))
 
 
+def test_decode_into_16_byte_aligned_output():
+    """Outputs aligned to 16 but not 32 bytes take the 16-byte-store variant."""
+    blob = table_set("learned_kv")
+    xb = inputs("kv", 700, seed=4)
+    blocks, _ = oracle.encode(blob, xb, nthreads=8)
+    t = ecco.Tables(blob, DEV)
+    flat = torch.zeros(700 * 128 + 8, dtype=torch.bfloat16, device=DEV)
+    out = flat[8:].view(700, 128)
+    assert out.data_ptr() % 32 == 16
+    ecco.decode(torch.from_numpy(blocks).to(DEV), t, out=out)
+    np.testing.assert_array_equal(bits(out), oracle.decode(blob, blocks, nthreads=8))
+    assert (bits(flat[:8]) == 0).all()
+
+
 def test_empty_inputs_enqueue_nothing():
     t = ecco.Tables(table_set("random0"), DEV)
     x = torch.empty(0, dtype=torch.bfloat16, device=DEV)
