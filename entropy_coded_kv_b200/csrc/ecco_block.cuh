@@ -88,7 +88,8 @@ __device__ __forceinline__ void refill(Stream& st, const uint32_t* ws, int strid
     }
 }
 
-// Decodes 8 symbols.  Returns their nibbles; `kv` = number of them that end
+// Decodes 8 symbols.  Returns their nibbles (symbol k in bits 4k..4k+3); `kv`
+// = number of them that end
 // at or before bit 512 (8 unless CHECK and the block clips here or earlier).
 template <bool CHECK>
 __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, const uint32_t* ws, int stride,
@@ -106,7 +107,7 @@ __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, cons
         for (int j = 0; j < 4; ++j) {
             uint32_t e = lut[cur & 0xffu];
             uint32_t len = e >> 4;
-            nib |= (e & 15u) << (4 * (4 * half + j));
+            nib = __funnelshift_r(nib, e, 4);  // symbol into the top nibble; the first ends at the bottom
             cur >>= len;
             u += (int)len;
             if (CHECK) kv += (used + u <= st.room) ? 1 : 0;

@@ -62,7 +62,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     uint32_t* ws = s_w + tid;
     const int64_t gpr = d.groups_per_row;
-    int64_t item = (int64_t)blockIdx.x * kDecThreads + tid;
+    // Item order: consecutive lanes take consecutive blocks; the warps of a
+    // round are spread over all CTAs first, so a partial last round is shared
+    // by every SM instead of loading the first few.
+    int64_t item = ((int64_t)(tid >> 5) * gridDim.x + blockIdx.x) * 32 + (tid & 31);
     int64_t r = item / gpr, g = item - r * gpr;
     for (; item < walk.total; item += (int64_t)gridDim.x * kDecThreads) {
         const uint8_t* src = blocks + (d.src_offset + r * d.src_row_stride + g) * ECCO_BLOCK_BYTES;
