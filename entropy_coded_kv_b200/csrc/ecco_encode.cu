@@ -1,4 +1,5 @@
-// Encoder: one warp per 128-value group, lane l owning values 4l..4l+3.
+// Encoder: 16 lanes per 128-value group (two groups per warp), lane l of a
+// half-warp owning values 8l..8l+7.
 //
 // Steps ("Ecco: Improving Memory Bandwidth and Capacity for LLMs via
 // Entropy-aware Cache Compression", review page):
@@ -14,177 +15,214 @@
 //   pad       spare bits filled with the largest remaining outliers, 15 bits
 //             each, at most 16 (free parameters: "Number of padded outlier slots").
 //
-// Every fp32 operation is an explicitly rounded intrinsic (__fmul_rn, __fadd_rn,
-// __fsub_rn, __fdiv_rn, __frcp_rn) so none is fused.  Tables are read through
-// the read-only data cache (all lanes of a warp read the same pattern row), so
-// a launch of a few thousand groups pays no per-CTA table staging.
+// Cost notes.  Per-group scalar work runs once per half-warp instruction, so
+// two groups share it.  The scale needs no divide per group: the code of
+// |x_m| / S_t is looked up by the bf16 magnitude of x_m, and s and 1/s by the
+// code, from tables the library builds on the device with the same IEEE
+// operations.  Thresholds, codeword lengths and codewords of one pattern share
+// one shared-memory row, so a symbol's position in the threshold search also
+// addresses its length and its codeword.  Every other fp32 operation is an
+// explicitly rounded intrinsic, so none is fused.
 #include "ecco_internal.cuh"
 
 namespace ecco {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kEncWarps = 8;  // warps per CTA
+constexpr int kEncWarps = 8;  // warps per CTA (16 groups in flight)
+constexpr int kRow = 97;      // words per pattern row: T[16] | lens4[16] | code[4][16] | pad
+constexpr int kRowLens = 16;
+constexpr int kRowCode = 32;
 
-struct Counters {  // warp-uniform
+struct Counters {  // uniform within a half-warp
     uint32_t groups, zero, clipped, padded, records, nonfinite;
     unsigned long long bits;
 };
 
-__device__ __forceinline__ uint32_t pick4(uint32_t a, uint32_t b, uint32_t c, uint32_t d, int j)
+__device__ __forceinline__ uint32_t hw_max(uint32_t m, uint32_t v) { return __reduce_max_sync(m, v); }
+__device__ __forceinline__ uint32_t hw_min(uint32_t m, uint32_t v) { return __reduce_min_sync(m, v); }
+__device__ __forceinline__ uint32_t hw_add(uint32_t m, uint32_t v) { return __reduce_add_sync(m, v); }
+
+__device__ __forceinline__ float hw_minf(uint32_t m, float v)
 {
-    uint32_t lo = (j & 1) ? b : a;
-    uint32_t hi = (j & 1) ? d : c;
-    return (j & 2) ? hi : lo;
+    float r;
+    asm volatile("redux.sync.min.f32 %0, %1, %2;" : "=f"(r) : "f"(v), "r"(m));
+    return r;
 }
 
-// Encodes the group at `src` into the block at `dst`.  All 32 lanes call it.
-__device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, uint32_t* buf, float S_t,
-                                             float2 endA, float2 endB, const uint16_t* src, uint8_t* dst,
-                                             int lane, Counters& cnt)
+__device__ __forceinline__ float hw_maxf(uint32_t m, float v)
 {
-    // ---- load 4 values (8 bytes per lane, 256 contiguous bytes per warp)
-    uint2 raw = __ldg(reinterpret_cast<const uint2*>(src) + lane);
-    uint32_t b0 = raw.x & 0xffffu, b1 = raw.x >> 16, b2 = raw.y & 0xffffu, b3 = raw.y >> 16;
-    const int i0 = 4 * lane;
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, %2;" : "=f"(r) : "f"(v), "r"(m));
+    return r;
+}
 
-    // ---- first index of the largest magnitude: key = |x| << 7 | (127 - i)
-    auto keyof = [&](uint32_t v, int i) { return ((v & 0x7fffu) << 7) | (uint32_t)(127 - i); };
-    uint32_t key = max(max(keyof(b0, i0), keyof(b1, i0 + 1)), max(keyof(b2, i0 + 2), keyof(b3, i0 + 3)));
-    key = __reduce_max_sync(kFull, key);
-    if ((key >> 7) >= 0x7f80u) {  // a NaN or Inf in the group: encode it as +0 and recount
-        int nf = 0;
-        if ((b0 & 0x7f80u) == 0x7f80u) { b0 = 0; ++nf; }
-        if ((b1 & 0x7f80u) == 0x7f80u) { b1 = 0; ++nf; }
-        if ((b2 & 0x7f80u) == 0x7f80u) { b2 = 0; ++nf; }
-        if ((b3 & 0x7f80u) == 0x7f80u) { b3 = 0; ++nf; }
-        cnt.nonfinite += __reduce_add_sync(kFull, (uint32_t)nf);
-        key = max(max(keyof(b0, i0), keyof(b1, i0 + 1)), max(keyof(b2, i0 + 2), keyof(b3, i0 + 3)));
-        key = __reduce_max_sync(kFull, key);
+// key = |x| << 8 | (127 - i) << 1 | sign: the largest key is the first index
+// of the largest magnitude, and it carries that element's sign.
+__device__ __forceinline__ uint32_t keyof(uint32_t v, int i)
+{
+    return ((v & 0x7fffu) << 8) | ((uint32_t)(127 - i) << 1) | (v >> 15);
+}
+
+__device__ __forceinline__ int quantise(const uint32_t* R, float t7, float v)
+{
+    int idx = (t7 < v) ? 8 : 0;
+    idx += (__uint_as_float(R[idx + 3]) < v) ? 4 : 0;
+    idx += (__uint_as_float(R[idx + 1]) < v) ? 2 : 0;
+    idx += (__uint_as_float(R[idx]) < v) ? 1 : 0;
+    return idx;
+}
+
+// Encodes one group with the 16 lanes of `gmask`; hl = lane within the half.
+__device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, const uint32_t* rows,
+                                             uint32_t* buf, const float2 (&ends)[4], const uint16_t* src,
+                                             uint8_t* dst, int hl, uint32_t gmask, Counters& cnt)
+{
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(src) + hl);
+    uint32_t b[8] = {q.x & 0xffffu, q.x >> 16, q.y & 0xffffu, q.y >> 16,
+                     q.z & 0xffffu, q.z >> 16, q.w & 0xffffu, q.w >> 16};
+    const int i0 = 8 * hl;
+
+    uint32_t key = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) key = max(key, keyof(b[j], i0 + j));
+    key = hw_max(gmask, key);
+    if ((key >> 8) >= 0x7f80u) {  // a NaN or Inf in the group: encoded as +0, counted
+        uint32_t nf = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if ((b[j] & 0x7f80u) == 0x7f80u) {
+                b[j] = 0;
+                ++nf;
+            }
+        cnt.nonfinite += hw_add(gmask, nf);
+        key = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) key = max(key, keyof(b[j], i0 + j));
+        key = hw_max(gmask, key);
     }
-    const int m = 127 - (int)(key & 127u);
-    const int mlane = m >> 2, mj = m & 3;
-    const uint32_t xm_bits = __shfl_sync(kFull, pick4(b0, b1, b2, b3, mj), mlane);
+    const int m = 127 - (int)((key >> 1) & 127u);
+    const bool owner = (hl == (m >> 3));
+    const int mj = m & 7;
 
-    // ---- group scale: E4M3(x_m / S_t), round-half-even, saturating
-    const float r = __fdiv_rn(bf16_bits_to_f32(xm_bits), S_t);
-    const uint32_t code = (uint32_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
-    const float fp8v = e4m3_to_f32(code);
+    // ---- group scale by table: E4M3(|x_m| / S_t) with x_m's sign; then 1/s
+    const uint32_t code = (uint32_t)__ldg(&tb->code_of_mag[key >> 8]) | ((key & 1u) << 7);
     cnt.groups += 1;
-    if (fp8v == 0.0f) {
-        if (lane < 16) reinterpret_cast<uint32_t*>(dst)[lane] = 0u;
+    if ((code & 0x7fu) == 0u) {
+        reinterpret_cast<uint32_t*>(dst)[hl] = 0u;
         cnt.zero += 1;
         return;
     }
-    const float s = __fmul_rn(S_t, fp8v);
-    const float inv = __frcp_rn(s);  // correctly rounded 1/s
+    const float inv = __ldg(&tb->inv_of_code[code]);
 
-    // ---- normalise; min / max over i != m (the scale element's slot takes the
-    // value of a neighbour from the same lane, which leaves both extremes alone)
-    float u0 = __fmul_rn(bf16_bits_to_f32(b0), inv), u1 = __fmul_rn(bf16_bits_to_f32(b1), inv);
-    float u2 = __fmul_rn(bf16_bits_to_f32(b2), inv), u3 = __fmul_rn(bf16_bits_to_f32(b3), inv);
-    float e0 = u0, e1 = u1, e2 = u2, e3 = u3;
-    if (lane == mlane) {
-        if (mj == 0) e0 = u1;
-        if (mj == 1) e1 = u0;
-        if (mj == 2) e2 = u3;
-        if (mj == 3) e3 = u2;
+    // ---- normalise; min / max over i != m (the scale element's slot takes a
+    // same-lane neighbour's value, which leaves both extremes alone)
+    float u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j] = __fmul_rn(bf16_bits_to_f32(b[j]), inv);
+    float lmin, lmax;
+    {
+        float e[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) e[j] = (owner && j == mj) ? u[j ^ 1] : u[j];
+        lmin = fminf(fminf(fminf(e[0], e[1]), fminf(e[2], e[3])), fminf(fminf(e[4], e[5]), fminf(e[6], e[7])));
+        lmax = fmaxf(fmaxf(fmaxf(e[0], e[1]), fmaxf(e[2], e[3])), fmaxf(fmaxf(e[4], e[5]), fmaxf(e[6], e[7])));
     }
-    const float umin = warp_min_f32(fminf(fminf(e0, e1), fminf(e2, e3)));
-    const float umax = warp_max_f32(fmaxf(fmaxf(e0, e1), fmaxf(e2, e3)));
+    const float umin = hw_minf(gmask, lmin);
+    const float umax = hw_maxf(gmask, lmax);
 
-    // ---- pattern: lane holds patterns lane and lane + 32
-    float d0 = __fsub_rn(umin, endA.x), d1 = __fsub_rn(umax, endA.y);
-    const float ea = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
-    d0 = __fsub_rn(umin, endB.x);
-    d1 = __fsub_rn(umax, endB.y);
-    const float eb = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
-    const bool takeB = eb < ea;
-    const uint32_t ebits = __float_as_uint(takeB ? eb : ea);  // e >= +0: bit order is value order
-    const uint32_t emin = __reduce_min_sync(kFull, ebits);
-    const int p = (int)__reduce_min_sync(kFull, ebits == emin ? (uint32_t)lane + (takeB ? 32u : 0u) : 64u);
-
-    // ---- quantise: number of thresholds strictly below u (branchless search)
-    const float* T = tb->T16[p];
-    const float t7 = __ldg(T + 7);
-    auto quant = [&](float v) {
-        int idx = (t7 < v) ? 8 : 0;
-        idx += (__ldg(T + idx + 3) < v) ? 4 : 0;
-        idx += (__ldg(T + idx + 1) < v) ? 2 : 0;
-        idx += (__ldg(T + idx) < v) ? 1 : 0;
-        return (uint32_t)idx;
-    };
-    uint32_t s0 = quant(u0), s1 = quant(u1), s2 = quant(u2), s3 = quant(u3);
-    if (lane == mlane) {
-        if (mj == 0) s0 = 15;
-        if (mj == 1) s1 = 15;
-        if (mj == 2) s2 = 15;
-        if (mj == 3) s3 = 15;
+    // ---- pattern: this lane evaluates patterns hl, hl+16, hl+32, hl+48
+    float best = INFINITY;
+    uint32_t bp = 64;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float d0 = __fsub_rn(umin, ends[k].x), d1 = __fsub_rn(umax, ends[k].y);
+        float e = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
+        if (e < best) {
+            best = e;
+            bp = (uint32_t)(hl + 16 * k);
+        }
     }
+    const uint32_t eb = __float_as_uint(best);  // e >= +0: bit order is value order
+    const uint32_t emin = hw_min(gmask, eb);
+    const int p = (int)hw_min(gmask, eb == emin ? bp : 64u);
 
-    // ---- codebook: total length per codebook (4 byte lanes), shortest wins
-    const uint32_t* L4 = tb->lens4[p];
-    const uint32_t acc = __ldg(L4 + s0) + __ldg(L4 + s1) + __ldg(L4 + s2) + __ldg(L4 + s3);
-    const uint32_t lo = __reduce_add_sync(kFull, acc & 0x00ff00ffu);         // h = 0, 2
-    const uint32_t hi = __reduce_add_sync(kFull, (acc >> 8) & 0x00ff00ffu);  // h = 1, 3
+    // ---- quantise (count of thresholds strictly below u); lengths
+    const uint32_t* R = rows + p * kRow;
+    const float t7 = __uint_as_float(R[7]);
+    int sym[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sym[j] = (owner && j == mj) ? 15 : quantise(R, t7, u[j]);
+    uint32_t acc = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc += R[kRowLens + sym[j]];
+    const uint32_t lo = hw_add(gmask, acc & 0x00ff00ffu);         // h = 0, 2
+    const uint32_t hi = hw_add(gmask, (acc >> 8) & 0x00ff00ffu);  // h = 1, 3
     int h = 0, L = (int)(lo & 0xffffu);
     if ((int)(hi & 0xffffu) < L) { L = (int)(hi & 0xffffu); h = 1; }
     if ((int)(lo >> 16) < L) { L = (int)(lo >> 16); h = 2; }
     if ((int)(hi >> 16) < L) { L = (int)(hi >> 16); h = 3; }
 
-    // ---- this lane's 4 codewords, concatenated in stream order (<= 32 bits)
-    const uint32_t* CW = tb->code[p][h];
-    const uint32_t c0 = __ldg(CW + s0), c1 = __ldg(CW + s1), c2 = __ldg(CW + s2), c3 = __ldg(CW + s3);
-    const int l0 = (int)(c0 >> 8), l1 = (int)(c1 >> 8), l2 = (int)(c2 >> 8), l3 = (int)(c3 >> 8);
-    uint32_t chunk = (c0 & 0xffu) | ((c1 & 0xffu) << l0);
-    chunk |= (c2 & 0xffu) << (l0 + l1);
-    chunk |= (c3 & 0xffu) << (l0 + l1 + l2);
-    const int clen = l0 + l1 + l2 + l3;
-    int off = clen;  // inclusive scan of chunk lengths
+    // ---- two chunks of 4 codewords each, in stream order (<= 32 bits each)
+    const uint32_t* CW = R + kRowCode + 16 * h;
+    uint32_t ch[2];
+    int cl[2];
 #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        int t = __shfl_up_sync(kFull, off, d);
-        if (lane >= d) off += t;
+    for (int c = 0; c < 2; ++c) {
+        uint32_t w = 0;
+        int n = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t e = CW[sym[4 * c + j]];
+            w |= (e & 0xffu) << n;
+            n += (int)(e >> 8);
+        }
+        ch[c] = w;
+        cl[c] = n;
     }
-    off -= clen;
+    const int tot = cl[0] + cl[1];
+    int off = tot;  // inclusive scan over the 16 lanes
+#pragma unroll
+    for (int dlt = 1; dlt < 16; dlt <<= 1) {
+        int t = __shfl_up_sync(gmask, off, dlt, 16);
+        if (hl >= dlt) off += t;
+    }
+    off -= tot;
 
     // ---- OR the chunks into the block; bits at or past 512 are dropped (clip)
-    const int bpos = kHdrBits + off;
-    const int w = bpos >> 5, sh = bpos & 31;
-    if (w < 16) atomicOr(&buf[w], chunk << sh);
-    if (sh != 0 && sh + clen > 32 && w + 1 < 16) atomicOr(&buf[w + 1], chunk >> (32 - sh));
-    if (lane == 0) atomicOr(&buf[0], code | ((uint32_t)p << 8) | ((uint32_t)h << 14));
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const int bpos = kHdrBits + off + (c ? cl[0] : 0);
+        const int w = bpos >> 5, sh = bpos & 31;
+        if (w < 16) atomicOr(&buf[w], ch[c] << sh);
+        if (sh != 0 && sh + cl[c] > 32 && w + 1 < 16) atomicOr(&buf[w + 1], ch[c] >> (32 - sh));
+    }
+    if (hl == 0) atomicOr(&buf[0], code | ((uint32_t)p << 8) | ((uint32_t)h << 14));
 
     // ---- outlier records in the spare bits of an unclipped block
     if (L <= kPayloadBits) {
         const int n = min(kMaxRec, (kPayloadBits - L) / kRecBits);
         if (n > 0) {
-            // lane-local candidates, largest first (the scale element excluded)
-            uint32_t k0 = keyof(b0, i0) + 1u, k1 = keyof(b1, i0 + 1) + 1u;
-            uint32_t k2 = keyof(b2, i0 + 2) + 1u, k3 = keyof(b3, i0 + 3) + 1u;
-            if (lane == mlane) {
-                if (mj == 0) k0 = 0;
-                if (mj == 1) k1 = 0;
-                if (mj == 2) k2 = 0;
-                if (mj == 3) k3 = 0;
-            }
-            // q for each of the lane's values: clamp(rint(u * 127), -127, 127)
-            auto qof = [](float u) {
-                float v = rintf(__fmul_rn(u, 127.0f));
-                return (uint32_t)(int)fminf(fmaxf(v, -127.0f), 127.0f) & 0xffu;
-            };
-            const uint32_t rec0 = (uint32_t)i0 | (qof(u0) << 7), rec1 = (uint32_t)(i0 + 1) | (qof(u1) << 7);
-            const uint32_t rec2 = (uint32_t)(i0 + 2) | (qof(u2) << 7), rec3 = (uint32_t)(i0 + 3) | (qof(u3) << 7);
+            uint32_t k[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) k[j] = (owner && j == mj) ? 0u : keyof(b[j], i0 + j) + 1u;
             int at = kHdrBits + L;
-            for (int k = 0; k < n; ++k, at += kRecBits) {
-                uint32_t mine = max(max(k0, k1), max(k2, k3));
-                uint32_t best = __reduce_max_sync(kFull, mine);
-                if (mine == best) {  // exactly one lane: keys are unique
-                    uint32_t rec;
-                    if (best == k0) { rec = rec0; k0 = 0; }
-                    else if (best == k1) { rec = rec1; k1 = 0; }
-                    else if (best == k2) { rec = rec2; k2 = 0; }
-                    else { rec = rec3; k3 = 0; }
+            for (int r = 0; r < n; ++r, at += kRecBits) {
+                uint32_t mine = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mine = max(mine, k[j]);
+                const uint32_t bestk = hw_max(gmask, mine);
+                if (mine == bestk) {  // exactly one lane: keys are unique
+                    float uv = u[0];
+                    int i = i0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (k[j] == bestk) {
+                            uv = u[j];
+                            i = i0 + j;
+                            k[j] = 0u;
+                        }
+                    float v = fminf(fmaxf(rintf(__fmul_rn(uv, 127.0f)), -127.0f), 127.0f);
+                    const uint32_t rec = (uint32_t)i | (((uint32_t)(int)v & 0xffu) << 7);
                     const int ww = at >> 5, ss = at & 31;
                     atomicOr(&buf[ww], rec << ss);
                     if (ss > 32 - kRecBits) atomicOr(&buf[ww + 1], rec >> (32 - ss));
@@ -199,35 +237,45 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, u
         cnt.bits += kPayloadBits;
     }
 
-    __syncwarp();
-    if (lane < 16) {
-        reinterpret_cast<uint32_t*>(dst)[lane] = buf[lane];
-        buf[lane] = 0u;
-    }
-    __syncwarp();
+    __syncwarp(gmask);
+    reinterpret_cast<uint32_t*>(dst)[hl] = buf[hl];
+    buf[hl] = 0u;
+    __syncwarp(gmask);
 }
 
 __global__ void __launch_bounds__(kEncWarps * 32)
     encode_kernel(const DevTables* __restrict__ tb, const uint16_t* __restrict__ x, ecco_desc d,
                   uint8_t* __restrict__ out, ecco_stats* __restrict__ stats, GridWalk walk)
 {
-    __shared__ uint32_t sbuf[kEncWarps][20];  // 16 block words + spill, per warp
+    __shared__ uint32_t rows[kNPat * kRow];
+    __shared__ uint32_t bufs[2 * kEncWarps][20];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (lane < 20) sbuf[warp][lane] = 0u;
-    const float2 endA = __ldg(&tb->ends[lane]);
-    const float2 endB = __ldg(&tb->ends[lane + 32]);
-    const float S_t = __ldg(&tb->S_t);
-    __syncwarp();
+    for (int i = tid; i < kNPat * kRow; i += blockDim.x) {
+        const int p = i / kRow, c = i - p * kRow;
+        uint32_t v = 0;
+        if (c < 16) v = __float_as_uint(tb->T16[p][c]);
+        else if (c < kRowCode) v = tb->lens4[p][c - kRowLens];
+        else if (c < kRowCode + 64) v = (&tb->code[p][0][0])[c - kRowCode];
+        rows[i] = v;
+    }
+    for (int i = tid; i < 2 * kEncWarps * 20; i += blockDim.x) (&bufs[0][0])[i] = 0u;
+    const int half = lane >> 4, hl = lane & 15;
+    const uint32_t gmask = 0xffffu << (16 * half);
+    float2 ends[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ends[k] = __ldg(&tb->ends[hl + 16 * k]);
+    __syncthreads();
 
     Counters cnt = {0, 0, 0, 0, 0, 0, 0ull};
+    uint32_t* buf = bufs[2 * warp + half];
     const int64_t gpr = d.groups_per_row;
-    int64_t item = (int64_t)blockIdx.x * kEncWarps + warp;
+    int64_t item = ((int64_t)blockIdx.x * kEncWarps + warp) * 2 + half;
     int64_t r = item / gpr, g = item - r * gpr;
-    const int64_t step = (int64_t)gridDim.x * kEncWarps;
+    const int64_t step = (int64_t)gridDim.x * kEncWarps * 2;
     for (; item < walk.total; item += step) {
         const uint16_t* src = x + (d.src_offset + r * d.src_row_stride + g) * kG;
         uint8_t* dst = out + (d.dst_offset + r * d.dst_row_stride + g) * ECCO_BLOCK_BYTES;
-        encode_group(tb, sbuf[warp], S_t, endA, endB, src, dst, lane, cnt);
+        encode_group(tb, rows, buf, ends, src, dst, hl, gmask, cnt);
         g += walk.stride_g;
         r += walk.stride_r;
         if (g >= gpr) {
@@ -235,7 +283,7 @@ __global__ void __launch_bounds__(kEncWarps * 32)
             r += 1;
         }
     }
-    if (stats && lane == 0 && cnt.groups) {  // counters are warp-uniform
+    if (stats && hl == 0 && cnt.groups) {
         atomicAdd(&stats->n_groups, (unsigned long long)cnt.groups);
         if (cnt.zero) atomicAdd(&stats->n_zero, (unsigned long long)cnt.zero);
         if (cnt.clipped) atomicAdd(&stats->n_clipped, (unsigned long long)cnt.clipped);
@@ -252,9 +300,9 @@ cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_de
                           uint8_t* blocks, ecco_stats* stats, cudaStream_t s)
 {
     const int64_t total = d.rows * d.groups_per_row;
-    const int per_cta = kEncWarps;
+    const int per_cta = 2 * kEncWarps;
     int64_t want = (total + per_cta - 1) / per_cta;
-    int64_t cap = (int64_t)device_sm_count() * 8;  // resident warps to hide latency
+    int64_t cap = (int64_t)device_sm_count() * 6;  // resident CTAs to hide latency
     int grid = (int)(want < cap ? want : cap);
     GridWalk walk;
     walk.total = total;

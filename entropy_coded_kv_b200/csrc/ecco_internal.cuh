@@ -40,6 +40,12 @@ struct DevTables {
     uint32_t lens4[kNPat][16];      // byte h = length of symbol s in codebook h
     uint32_t code[kNPat][kNBook][16];  // bits 0-7 codeword in stream order, bits 8-11 length
     uint8_t lut[kNBook * kNPat][256];  // [h * 64 + p] (= header bits 8-15): next 8 stream bits -> symbol | length << 4
+    // Scale tables, filled on the device at creation with the same operations
+    // the encoder would otherwise run per group (IEEE divide, E4M3 rounding,
+    // fp32 multiply, correctly rounded reciprocal):
+    float s_of_code[256];           // S_t * fp8(code); 0 for zero and NaN codes
+    float inv_of_code[256];         // 1 / s_of_code (0 where s is 0)
+    uint8_t code_of_mag[32768];     // E4M3(|x| / S_t), saturating, for every bf16 magnitude |x|
 };
 
 }  // namespace ecco

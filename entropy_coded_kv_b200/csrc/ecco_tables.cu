@@ -108,6 +108,26 @@ void derive(const Blob& b, DevTables* t)
     }
 }
 
+// One thread per bf16 magnitude (32768) and per scale code (256).
+__global__ void scale_tables_kernel(DevTables* t)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const float S_t = t->S_t;
+    if (i < 32768) {
+        float r = __fdiv_rn(__uint_as_float((uint32_t)i << 16), S_t);
+        t->code_of_mag[i] = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+    }
+    if (i < 256) {
+        float s = 0.0f, inv = 0.0f;
+        if (!scale_code_is_null((uint32_t)i)) {
+            s = __fmul_rn(S_t, e4m3_to_f32((uint32_t)i));
+            inv = __frcp_rn(s);
+        }
+        t->s_of_code[i] = s;
+        t->inv_of_code[i] = inv;
+    }
+}
+
 }  // namespace
 
 extern "C" int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables** out)
@@ -135,6 +155,11 @@ extern "C" int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables**
     }
     cudaError_t e = cudaMemcpy(d, host, sizeof(DevTables), cudaMemcpyHostToDevice);
     delete host;
+    if (e == cudaSuccess) {
+        scale_tables_kernel<<<32768 / 256, 256>>>(d);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    }
     if (e != cudaSuccess) {
         cudaFree(d);
         return ECCO_ERR_CUDA;
