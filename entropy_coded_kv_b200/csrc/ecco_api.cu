@@ -145,31 +145,3 @@ extern "C" const char* ecco_strerror(int code)
 
 extern "C" int ecco_abi_version(void) { return 1; }
 
-namespace ecco {
-
-// Segments run back to back on the stream, one launch each.
-cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s)
-{
-    for (int i = 0; i < n; ++i) {
-        const ecco_desc& d = segs[i].desc;
-        if (d.rows == 0 || d.groups_per_row == 0) continue;
-        cudaError_t e = launch_decode(segs[i].tables, static_cast<const uint8_t*>(segs[i].src), d,
-                                      static_cast<uint16_t*>(segs[i].dst), s);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
-cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats, cudaStream_t s)
-{
-    for (int i = 0; i < n; ++i) {
-        const ecco_desc& d = segs[i].desc;
-        if (d.rows == 0 || d.groups_per_row == 0) continue;
-        cudaError_t e = launch_encode(segs[i].tables, static_cast<const uint16_t*>(segs[i].src), d,
-                                      static_cast<uint8_t*>(segs[i].dst), stats, s);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
-}  // namespace ecco

@@ -39,112 +39,175 @@ __device__ __forceinline__ void store16(uint16_t* dst, const uint32_t a[4], cons
     }
 }
 
-template <bool WIDE>
-__global__ void __launch_bounds__(kDecThreads, 1)
-    decode_kernel(const DevTables* __restrict__ tb, const uint8_t* __restrict__ blocks, ecco_desc d,
-                  uint16_t* __restrict__ y, GridWalk walk)
+// One tensor's share of a launch: its tables, buffers, descriptor, and where
+// its blocks start in the launch's concatenated block index.
+struct DecSeg {
+    const DevTables* tb;
+    const uint8_t* src;
+    uint16_t* dst;
+    ecco_desc d;
+    int64_t begin, count;
+};
+
+// Passed by value (a __grid_constant__ kernel parameter): no device-side
+// segment table has to be allocated or copied.
+template <int MAXSEG>
+struct DecParams {
+    int n_seg;
+    int64_t total;
+    DecSeg seg[MAXSEG];
+};
+
+// Each CTA decodes one contiguous, equal share of all blocks of the launch,
+// segment by segment, restaging the segment's tables in shared memory when
+// its share crosses into the next segment.
+template <bool WIDE, int MAXSEG>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecParams<MAXSEG> P)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kDecSmemLut);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kDecSmemLut + kDecSmemCt);
     const int tid = threadIdx.x;
-    {
-        const uint4* a = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
-        uint4* b = reinterpret_cast<uint4*>(s_lut);
-        for (int i = tid; i < (int)(kDecSmemLut / 16); i += kDecThreads) b[i] = a[i];
-        const uint4* c = reinterpret_cast<const uint4*>(&tb->Ct[0][0]);
-        uint4* e = reinterpret_cast<uint4*>(s_Ct);
-        for (int i = tid; i < (int)(kDecSmemCt / 16); i += kDecThreads) e[i] = c[i];
-    }
-    const float S_t = tb->S_t;
-    __syncthreads();
-
     uint32_t* ws = s_w + tid;
-    const int64_t gpr = d.groups_per_row;
-    // Item order: consecutive lanes take consecutive blocks; the warps of a
-    // round are spread over all CTAs first, so a partial last round is shared
-    // by every SM instead of loading the first few.
-    int64_t item = ((int64_t)(tid >> 5) * gridDim.x + blockIdx.x) * 32 + (tid & 31);
-    int64_t r = item / gpr, g = item - r * gpr;
-    for (; item < walk.total; item += (int64_t)gridDim.x * kDecThreads) {
-        const uint8_t* src = blocks + (d.src_offset + r * d.src_row_stride + g) * ECCO_BLOCK_BYTES;
-        uint16_t* dst = y + (d.dst_offset + r * d.dst_row_stride + g) * kG;
-        g += walk.stride_g;
-        r += walk.stride_r;
-        if (g >= gpr) {
-            g -= gpr;
-            r += 1;
-        }
 
-        uint4 q0 = ldg_nc_v4(src), q1 = ldg_nc_v4(src + 16), q2 = ldg_nc_v4(src + 32),
-              q3 = ldg_nc_v4(src + 48);
-        const uint32_t code = q0.x & 0xffu;
-        if (scale_code_is_null(code)) {
-            const uint32_t z[4] = {0u, 0u, 0u, 0u};
+    const int64_t share = (P.total + gridDim.x - 1) / gridDim.x;
+    int64_t lo = (int64_t)blockIdx.x * share;
+    const int64_t hi = min(P.total, lo + share);
+    for (int si = 0; si < P.n_seg && lo < hi; ++si) {
+        const DecSeg& S = P.seg[si];
+        const int64_t seg_end = S.begin + S.count;
+        if (seg_end <= lo) continue;
+        const int64_t stop = min(hi, seg_end);
+        const DevTables* tb = S.tb;
+        __syncthreads();  // the previous segment's tables are no longer read
+        {
+            const uint4* a = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
+            uint4* b = reinterpret_cast<uint4*>(s_lut);
+            for (int i = tid; i < (int)(kDecSmemLut / 16); i += kDecThreads) b[i] = a[i];
+            const uint4* c = reinterpret_cast<const uint4*>(&tb->Ct[0][0]);
+            uint4* e = reinterpret_cast<uint4*>(s_Ct);
+            for (int i = tid; i < (int)(kDecSmemCt / 16); i += kDecThreads) e[i] = c[i];
+        }
+        const float S_t = tb->S_t;
+        __syncthreads();
+
+        // local group index within the segment; consecutive threads take
+        // consecutive groups, kDecThreads per round
+        const int64_t gpr = S.d.groups_per_row;
+        const int64_t stride_r = kDecThreads / gpr, stride_g = kDecThreads % gpr;
+        int64_t item = lo - S.begin + tid;
+        const int64_t end = stop - S.begin;
+        int64_t r = item / gpr, g = item - r * gpr;
+        for (; item < end; item += kDecThreads) {
+            const uint8_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * ECCO_BLOCK_BYTES;
+            uint16_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * kG;
+            g += stride_g;
+            r += stride_r;
+            if (g >= gpr) {
+                g -= gpr;
+                r += 1;
+            }
+
+            uint4 q0 = ldg_nc_v4(src), q1 = ldg_nc_v4(src + 16), q2 = ldg_nc_v4(src + 32),
+                  q3 = ldg_nc_v4(src + 48);
+            const uint32_t code = q0.x & 0xffu;
+            if (scale_code_is_null(code)) {
+                const uint32_t z[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int k = 0; k < 8; ++k) store16<WIDE>(dst + 16 * k, z, z);
-            continue;
-        }
-        stage_words(ws, kWordStride, q0, q1, q2, q3);
-        const int p = (int)((q0.x >> 8) & 63u);
-        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;  // table h * 64 + p
-        const float s = __fmul_rn(S_t, e4m3_to_f32(code));
-        const ValuePlanes vp = make_planes(s, s_Ct, p);
+                for (int k = 0; k < 8; ++k) store16<WIDE>(dst + 16 * k, z, z);
+                continue;
+            }
+            stage_words(ws, kWordStride, q0, q1, q2, q3);
+            const int p = (int)((q0.x >> 8) & 63u);
+            const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;  // table h * 64 + p
+            const float s = __fmul_rn(S_t, e4m3_to_f32(code));
+            const ValuePlanes vp = make_planes(s, s_Ct, p);
 
-        Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
+            Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {  // 8 x 16 symbols, one 32-byte store each
-            uint32_t wa[4], wb[4];
-            chunk_values(st, lut, ws, kWordStride, vp, wa);
-            chunk_values(st, lut, ws, kWordStride, vp, wb);
-            store16<WIDE>(dst + 16 * c, wa, wb);
-        }
+            for (int c = 0; c < 8; ++c) {  // 8 x 16 symbols, one 32-byte store each
+                uint32_t wa[4], wb[4];
+                chunk_values(st, lut, ws, kWordStride, vp, wa);
+                chunk_values(st, lut, ws, kWordStride, vp, wb);
+                store16<WIDE>(dst + 16 * c, wa, wb);
+            }
 
-        if (st.room >= 0) {  // unclipped: outlier records follow the codewords
-            const int n = min(kMaxRec, st.room / kRecBits);
-            int at = kBlockBits - st.room;
-            for (int k = 0; k < n; ++k, at += kRecBits) {
-                uint32_t rec = read_record(ws, kWordStride, at);
-                int i = (int)(rec & 127u);
-                int qv = (int)(int8_t)(uint8_t)(rec >> 7);
-                float o = __fdiv_rn((float)qv, 127.0f);
-                dst[i] = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
+            if (st.room >= 0) {  // unclipped: outlier records follow the codewords
+                const int n = min(kMaxRec, st.room / kRecBits);
+                int at = kBlockBits - st.room;
+                for (int k = 0; k < n; ++k, at += kRecBits) {
+                    uint32_t rec = read_record(ws, kWordStride, at);
+                    int i = (int)(rec & 127u);
+                    int qv = (int)(int8_t)(uint8_t)(rec >> 7);
+                    float o = __fdiv_rn((float)qv, 127.0f);
+                    dst[i] = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
+                }
             }
         }
+        lo = stop;
     }
 }
+
+template <bool WIDE, int MAXSEG>
+cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
+{
+    static int configured = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured != dev) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<WIDE, MAXSEG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmem);
+        if (e != cudaSuccess) return e;
+        configured = dev;
+    }
+    int64_t want = (P.total + kDecThreads - 1) / kDecThreads;
+    int64_t cap = device_sm_count();
+    int grid = (int)(want < cap ? want : cap);
+    decode_kernel<WIDE, MAXSEG><<<grid, kDecThreads, kDecSmem, s>>>(P);
+    return cudaGetLastError();
+}
+
+bool wide_ok(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 }  // namespace
 
 cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
                           uint16_t* y, cudaStream_t s)
 {
-    static int configured_dev = -1;
-    int dev = t->device;
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kDecSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kDecSmem);
+    DecParams<1> P;
+    P.n_seg = 1;
+    P.total = d.rows * d.groups_per_row;
+    P.seg[0] = DecSeg{t->d, blocks, y, d, 0, P.total};
+    return wide_ok(y) ? run_decode<true, 1>(P, s) : run_decode<false, 1>(P, s);
+}
+
+// Segments are packed into launches of at most kMultiSeg; empty ones are skipped.
+cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s)
+{
+    constexpr int kMultiSeg = 64;
+    int i = 0;
+    while (i < n) {
+        DecParams<kMultiSeg> P;
+        P.n_seg = 0;
+        P.total = 0;
+        bool wide = true;
+        while (i < n && P.n_seg < kMultiSeg) {
+            const ecco_desc& d = segs[i].desc;
+            const int64_t cnt = d.rows * d.groups_per_row;
+            if (cnt > 0) {
+                P.seg[P.n_seg++] = DecSeg{segs[i].tables->d, static_cast<const uint8_t*>(segs[i].src),
+                                          static_cast<uint16_t*>(segs[i].dst), d, P.total, cnt};
+                P.total += cnt;
+                wide = wide && wide_ok(segs[i].dst);
+            }
+            ++i;
+        }
+        if (P.n_seg == 0) break;
+        cudaError_t e = wide ? run_decode<true, kMultiSeg>(P, s) : run_decode<false, kMultiSeg>(P, s);
         if (e != cudaSuccess) return e;
-        configured_dev = dev;
     }
-    const int64_t total = d.rows * d.groups_per_row;
-    int64_t want = (total + kDecThreads - 1) / kDecThreads;
-    int64_t cap = device_sm_count();
-    int grid = (int)(want < cap ? want : cap);
-    GridWalk walk;
-    walk.total = total;
-    int64_t stride = (int64_t)grid * kDecThreads;
-    walk.stride_r = stride / d.groups_per_row;
-    walk.stride_g = stride % d.groups_per_row;
-    if ((reinterpret_cast<uintptr_t>(y) & 31u) == 0)
-        decode_kernel<true><<<grid, kDecThreads, kDecSmem, s>>>(t->d, blocks, d, y, walk);
-    else
-        decode_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(t->d, blocks, d, y, walk);
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace ecco

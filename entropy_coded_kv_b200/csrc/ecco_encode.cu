@@ -131,13 +131,15 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     const float umax = hw_maxf(gmask, lmax);
 
     // ---- pattern: this lane evaluates patterns hl, hl+16, hl+32, hl+48
-    float best = INFINITY;
-    uint32_t bp = 64;
+    // (the first of the lane's patterns is taken unconditionally, so a group
+    // whose errors are all +inf still gets the lowest index, as scanning does)
+    float best = 0.0f;
+    uint32_t bp = (uint32_t)hl;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         float d0 = __fsub_rn(umin, ends[k].x), d1 = __fsub_rn(umax, ends[k].y);
         float e = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
-        if (e < best) {
+        if (k == 0 || e < best) {
             best = e;
             bp = (uint32_t)(hl + 16 * k);
         }
@@ -243,46 +245,79 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     __syncwarp(gmask);
 }
 
-__global__ void __launch_bounds__(kEncWarps * 32)
-    encode_kernel(const DevTables* __restrict__ tb, const uint16_t* __restrict__ x, ecco_desc d,
-                  uint8_t* __restrict__ out, ecco_stats* __restrict__ stats, GridWalk walk)
+struct EncSeg {
+    const DevTables* tb;
+    const uint16_t* src;
+    uint8_t* dst;
+    ecco_desc d;
+    int64_t begin, count;
+};
+
+template <int MAXSEG>
+struct EncParams {  // by value: no device-side segment table
+    int n_seg;
+    int64_t total;
+    ecco_stats* stats;
+    EncSeg seg[MAXSEG];
+};
+
+// Each CTA encodes one contiguous, equal share of all groups of the launch,
+// segment by segment, restaging the pattern rows when it enters a new segment.
+template <int MAXSEG>
+__global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_constant__ EncParams<MAXSEG> P)
 {
     __shared__ uint32_t rows[kNPat * kRow];
     __shared__ uint32_t bufs[2 * kEncWarps][20];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int i = tid; i < kNPat * kRow; i += blockDim.x) {
-        const int p = i / kRow, c = i - p * kRow;
-        uint32_t v = 0;
-        if (c < 16) v = __float_as_uint(tb->T16[p][c]);
-        else if (c < kRowCode) v = tb->lens4[p][c - kRowLens];
-        else if (c < kRowCode + 64) v = (&tb->code[p][0][0])[c - kRowCode];
-        rows[i] = v;
-    }
     for (int i = tid; i < 2 * kEncWarps * 20; i += blockDim.x) (&bufs[0][0])[i] = 0u;
     const int half = lane >> 4, hl = lane & 15;
     const uint32_t gmask = 0xffffu << (16 * half);
-    float2 ends[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) ends[k] = __ldg(&tb->ends[hl + 16 * k]);
-    __syncthreads();
-
-    Counters cnt = {0, 0, 0, 0, 0, 0, 0ull};
     uint32_t* buf = bufs[2 * warp + half];
-    const int64_t gpr = d.groups_per_row;
-    int64_t item = ((int64_t)blockIdx.x * kEncWarps + warp) * 2 + half;
-    int64_t r = item / gpr, g = item - r * gpr;
-    const int64_t step = (int64_t)gridDim.x * kEncWarps * 2;
-    for (; item < walk.total; item += step) {
-        const uint16_t* src = x + (d.src_offset + r * d.src_row_stride + g) * kG;
-        uint8_t* dst = out + (d.dst_offset + r * d.dst_row_stride + g) * ECCO_BLOCK_BYTES;
-        encode_group(tb, rows, buf, ends, src, dst, hl, gmask, cnt);
-        g += walk.stride_g;
-        r += walk.stride_r;
-        if (g >= gpr) {
-            g -= gpr;
-            r += 1;
+    Counters cnt = {0, 0, 0, 0, 0, 0, 0ull};
+
+    const int64_t share = (P.total + gridDim.x - 1) / gridDim.x;
+    int64_t lo = (int64_t)blockIdx.x * share;
+    const int64_t hi = min(P.total, lo + share);
+    for (int si = 0; si < P.n_seg && lo < hi; ++si) {
+        const EncSeg& S = P.seg[si];
+        const int64_t seg_end = S.begin + S.count;
+        if (seg_end <= lo) continue;
+        const int64_t stop = min(hi, seg_end);
+        const DevTables* tb = S.tb;
+        __syncthreads();  // the previous segment's rows are no longer read
+        for (int i = tid; i < kNPat * kRow; i += blockDim.x) {
+            const int p = i / kRow, c = i - p * kRow;
+            uint32_t v = 0;
+            if (c < 16) v = __float_as_uint(tb->T16[p][c]);
+            else if (c < kRowCode) v = tb->lens4[p][c - kRowLens];
+            else if (c < kRowCode + 64) v = (&tb->code[p][0][0])[c - kRowCode];
+            rows[i] = v;
         }
+        float2 ends[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ends[k] = __ldg(&tb->ends[hl + 16 * k]);
+        __syncthreads();
+
+        constexpr int kPerRound = 2 * kEncWarps;  // groups per CTA round
+        const int64_t gpr = S.d.groups_per_row;
+        const int64_t stride_r = kPerRound / gpr, stride_g = kPerRound % gpr;
+        int64_t item = lo - S.begin + 2 * warp + half;
+        const int64_t end = stop - S.begin;
+        int64_t r = item / gpr, g = item - r * gpr;
+        for (; item < end; item += kPerRound) {
+            const uint16_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * kG;
+            uint8_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * ECCO_BLOCK_BYTES;
+            encode_group(tb, rows, buf, ends, src, dst, hl, gmask, cnt);
+            g += stride_g;
+            r += stride_r;
+            if (g >= gpr) {
+                g -= gpr;
+                r += 1;
+            }
+        }
+        lo = stop;
     }
+    ecco_stats* stats = P.stats;
     if (stats && hl == 0 && cnt.groups) {
         atomicAdd(&stats->n_groups, (unsigned long long)cnt.groups);
         if (cnt.zero) atomicAdd(&stats->n_zero, (unsigned long long)cnt.zero);
@@ -294,23 +329,55 @@ __global__ void __launch_bounds__(kEncWarps * 32)
     }
 }
 
+template <int MAXSEG>
+cudaError_t run_encode(const EncParams<MAXSEG>& P, cudaStream_t s)
+{
+    const int per_cta = 2 * kEncWarps;
+    int64_t want = (P.total + per_cta - 1) / per_cta;
+    int64_t cap = (int64_t)device_sm_count() * 3;  // resident CTAs at 3 per SM
+    int grid = (int)(want < cap ? want : cap);
+    encode_kernel<MAXSEG><<<grid, kEncWarps * 32, 0, s>>>(P);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
                           uint8_t* blocks, ecco_stats* stats, cudaStream_t s)
 {
-    const int64_t total = d.rows * d.groups_per_row;
-    const int per_cta = 2 * kEncWarps;
-    int64_t want = (total + per_cta - 1) / per_cta;
-    int64_t cap = (int64_t)device_sm_count() * 6;  // resident CTAs to hide latency
-    int grid = (int)(want < cap ? want : cap);
-    GridWalk walk;
-    walk.total = total;
-    int64_t stride = (int64_t)grid * per_cta;
-    walk.stride_r = stride / d.groups_per_row;
-    walk.stride_g = stride % d.groups_per_row;
-    encode_kernel<<<grid, kEncWarps * 32, 0, s>>>(t->d, x, d, blocks, stats, walk);
-    return cudaGetLastError();
+    EncParams<1> P;
+    P.n_seg = 1;
+    P.total = d.rows * d.groups_per_row;
+    P.stats = stats;
+    P.seg[0] = EncSeg{t->d, x, blocks, d, 0, P.total};
+    return run_encode<1>(P, s);
+}
+
+// Segments are packed into launches of at most kMultiSeg; empty ones are skipped.
+cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats, cudaStream_t s)
+{
+    constexpr int kMultiSeg = 64;
+    int i = 0;
+    while (i < n) {
+        EncParams<kMultiSeg> P;
+        P.n_seg = 0;
+        P.total = 0;
+        P.stats = stats;
+        while (i < n && P.n_seg < kMultiSeg) {
+            const ecco_desc& d = segs[i].desc;
+            const int64_t cnt = d.rows * d.groups_per_row;
+            if (cnt > 0) {
+                P.seg[P.n_seg++] = EncSeg{segs[i].tables->d, static_cast<const uint16_t*>(segs[i].src),
+                                          static_cast<uint8_t*>(segs[i].dst), d, P.total, cnt};
+                P.total += cnt;
+            }
+            ++i;
+        }
+        if (P.n_seg == 0) break;
+        cudaError_t e = run_encode<kMultiSeg>(P, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace ecco

@@ -58,10 +58,6 @@ struct ecco_tables {
 namespace ecco {
 
 // ------------------------------------------------------------ launchers
-struct GridWalk {  // 2-D group index walked with a fixed stride
-    int64_t total;
-    int64_t stride_r, stride_g;  // (gridDim*items per CTA) / gpr, % gpr
-};
 
 cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
                           uint8_t* blocks, ecco_stats* stats, cudaStream_t s);

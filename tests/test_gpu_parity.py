@@ -331,3 +331,36 @@ def test_full_size_mlp_weight_sampled():
         rsel = sample_rows(rows, 96, batch)
         bl = blocks.view(rows, cols // 128, 64)[torch.from_numpy(rsel).to(DEV)].cpu().numpy()
         gemv_check(blob, bl, len(rsel), cols, bits(x), yv[:, rsel])
+
+
+def test_multi_segment_many_small_segments_cross_launches():
+    """70 segments (more than one launch's worth), some empty, mixed tables and
+    sizes, so CTA shares cross segment boundaries mid-round."""
+    names = ["learned_kv", "random1", "learned_w", "random0"]
+    tabs = {n: ecco.Tables(table_set(n), DEV) for n in names}
+    rng = np.random.default_rng(70)
+    plan = []
+    for i in range(70):
+        n = int(rng.choice([0, 1, 7, 33, 130, 1500]))
+        plan.append((names[i % 4], n, i))
+    segs, outs, xs = [], [], []
+    for name, n, i in plan:
+        xb = inputs(["kv", "gauss", "t5", "c1"][i % 4], max(n, 1), seed=1000 + i)[: n * 128]
+        x = to_dev_bf16(xb) if n else torch.empty(0, dtype=torch.bfloat16, device=DEV)
+        o = torch.empty((n, 64), dtype=torch.uint8, device=DEV)
+        segs.append(ecco.Seg(tabs[name], x, o))
+        outs.append(o)
+        xs.append(xb)
+    st = ecco.new_stats(DEV)
+    ecco.encode_multi(segs, st)
+    ys = [torch.empty((o.shape[0], 128), dtype=torch.bfloat16, device=DEV) for o in outs]
+    ecco.decode_multi([ecco.Seg(tabs[name], o, y) for (name, _, _), o, y in zip(plan, outs, ys)])
+    tot = 0
+    for (name, n, _), xb, o, y in zip(plan, xs, outs, ys):
+        if n == 0:
+            continue
+        want, wst = oracle.encode(table_set(name), xb, nthreads=4)
+        np.testing.assert_array_equal(o.cpu().numpy(), want)
+        np.testing.assert_array_equal(bits(y).reshape(-1, 128), oracle.decode(table_set(name), want, nthreads=4))
+        tot += wst.n_groups
+    assert ecco.read_stats(st)["n_groups"] == tot
