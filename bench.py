@@ -704,14 +704,27 @@ def main():
         dist.destroy_process_group()
 
 
+def source_hash() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "entropy_coded_kv_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_for(workload, kernel):
-    """DRAM bytes per launch from the committed ncu summary, if one matches."""
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    or None when no capture matches or the kernel sources changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    return d.get(f"{workload}:{kernel}")
+    if d.get("source_hash") != source_hash():
+        return None
+    return d.get(f"{workload}:{kernel.split()[0]}")
 
 
 def run_reference(args, world):
