@@ -21,7 +21,7 @@ MAX_SEGMENTS = 256
 EXPORTED = [
     "ecco_tables_create", "ecco_tables_destroy", "ecco_select_encode", "ecco_decode",
     "ecco_decode_gemv", "ecco_decode_multi", "ecco_encode_multi", "ecco_strerror",
-    "ecco_abi_version",
+    "ecco_abi_version", "ecco_device_timeouts",
 ]
 
 
@@ -66,6 +66,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_strerror.argtypes = [I]
     L.ecco_strerror.restype = ctypes.c_char_p
     L.ecco_abi_version.argtypes = []
+    L.ecco_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     for fn in EXPORTED:
         if fn != "ecco_strerror":
             getattr(L, fn).restype = I

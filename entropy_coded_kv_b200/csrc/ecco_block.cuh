@@ -176,6 +176,33 @@ __device__ __forceinline__ void stage_words(uint32_t* ws, int stride, const uint
     ws[15 * stride] = q3.w;
 }
 
+// Copies a tensor's decode tables (65,536 B) and transposed centroids (4,096 B)
+// into shared memory with every 16-byte load issued before any store.
+template <int NT>
+__device__ __forceinline__ void stage_tables(const DevTables* tb, uint8_t* s_lut, float* s_Ct, int tid)
+{
+    constexpr int kLutVec = (int)(sizeof(((DevTables*)0)->lut) / 16);
+    constexpr int kCtVec = (int)(sizeof(((DevTables*)0)->Ct) / 16);
+    constexpr int kAll = kLutVec + kCtVec;
+    constexpr int kPer = (kAll + NT - 1) / NT;
+    const uint4* lut = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
+    const uint4* ct = reinterpret_cast<const uint4*>(&tb->Ct[0][0]);
+    uint4 v[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = tid + k * NT;
+        if (i < kAll) v[k] = __ldg(i < kLutVec ? lut + i : ct + (i - kLutVec));
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = tid + k * NT;
+        if (i < kLutVec)
+            reinterpret_cast<uint4*>(s_lut)[i] = v[k];
+        else if (i < kAll)
+            reinterpret_cast<uint4*>(s_Ct)[i - kLutVec] = v[k];
+    }
+}
+
 __device__ __forceinline__ void stg256(void* p, const uint32_t a[4], const uint32_t b[4])
 {
     asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a[0]), "r"(a[1]),

@@ -81,14 +81,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         const int64_t stop = min(hi, seg_end);
         const DevTables* tb = S.tb;
         __syncthreads();  // the previous segment's tables are no longer read
-        {
-            const uint4* a = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
-            uint4* b = reinterpret_cast<uint4*>(s_lut);
-            for (int i = tid; i < (int)(kDecSmemLut / 16); i += kDecThreads) b[i] = a[i];
-            const uint4* c = reinterpret_cast<const uint4*>(&tb->Ct[0][0]);
-            uint4* e = reinterpret_cast<uint4*>(s_Ct);
-            for (int i = tid; i < (int)(kDecSmemCt / 16); i += kDecThreads) e[i] = c[i];
-        }
+        stage_tables<kDecThreads>(tb, s_lut, s_Ct, tid);
         const float S_t = tb->S_t;
         __syncthreads();
 

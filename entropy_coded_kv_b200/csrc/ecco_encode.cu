@@ -285,13 +285,28 @@ __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_
         const int64_t stop = min(hi, seg_end);
         const DevTables* tb = S.tb;
         __syncthreads();  // the previous segment's rows are no longer read
-        for (int i = tid; i < kNPat * kRow; i += blockDim.x) {
-            const int p = i / kRow, c = i - p * kRow;
-            uint32_t v = 0;
-            if (c < 16) v = __float_as_uint(tb->T16[p][c]);
-            else if (c < kRowCode) v = tb->lens4[p][c - kRowLens];
-            else if (c < kRowCode + 64) v = (&tb->code[p][0][0])[c - kRowCode];
-            rows[i] = v;
+        {
+            // 24 16-byte pieces per pattern row (thresholds, lengths, codewords),
+            // all loads issued before any store so the copy costs one latency.
+            constexpr int kRowVec = 24, kPer = kNPat * kRowVec / (kEncWarps * 32);
+            uint4 v[kPer];
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int i = tid + k * kEncWarps * 32, p = i / kRowVec, part = i - p * kRowVec;
+                const uint4* src = part < 4   ? reinterpret_cast<const uint4*>(tb->T16[p]) + part
+                                   : part < 8 ? reinterpret_cast<const uint4*>(tb->lens4[p]) + (part - 4)
+                                              : reinterpret_cast<const uint4*>(&tb->code[p][0][0]) + (part - 8);
+                v[k] = __ldg(src);
+            }
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int i = tid + k * kEncWarps * 32, p = i / kRowVec, part = i - p * kRowVec;
+                uint32_t* d = rows + p * kRow + 4 * part;  // T at 0..15, lengths 16..31, codewords 32..95
+                d[0] = v[k].x;
+                d[1] = v[k].y;
+                d[2] = v[k].z;
+                d[3] = v[k].w;
+            }
         }
         float2 ends[4];
 #pragma unroll

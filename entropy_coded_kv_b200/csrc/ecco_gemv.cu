@@ -1,4 +1,5 @@
-// Fused decode + matrix-vector product on CUDA cores.
+// Fused decode + matrix-vector product on CUDA cores (batch 1..4; larger
+// batches go to the tensor-core kernel in ecco_gemm_tc.cu).
 //
 // y[b][r] = sum_k W~[r][k] * x[b][k], W~ the decoded matrix, never written to
 // memory (the review page's figure list: "Normalized Memory Requests for a
@@ -50,12 +51,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const int64_t g0 = (int64_t)blockIdx.y * kGvColGroups;
     const int ng = (int)min((int64_t)kGvColGroups, gpr - g0);
     {
-        const uint4* a = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
-        uint4* b = reinterpret_cast<uint4*>(s_lut);
-        for (int i = tid; i < (int)(kGvLut / 16); i += kGvThreads) b[i] = a[i];
-        const uint4* c = reinterpret_cast<const uint4*>(&tb->Ct[0][0]);
-        uint4* e = reinterpret_cast<uint4*>(s_Ct);
-        for (int i = tid; i < (int)(kGvCt / 16); i += kGvThreads) e[i] = c[i];
+        stage_tables<kGvThreads>(tb, s_lut, s_Ct, tid);
         for (int i = tid; i < kGvColGroups * kG * B; i += kGvThreads) {
             int k = i / B, bb = i - k * B;
             float v = 0.0f;
@@ -163,7 +159,7 @@ cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t row
 {
     if (batch == 1) return run_gemv<1>(t, blocks, rows, cols, x, batch, y, s);
     if (batch <= 4) return run_gemv<4>(t, blocks, rows, cols, x, batch, y, s);
-    return run_gemv<16>(t, blocks, rows, cols, x, batch, y, s);
+    return launch_gemm_tc(t, blocks, rows, cols, x, batch, y, s);  // tensor cores, ecco_gemm_tc.cu
 }
 
 }  // namespace ecco

@@ -65,6 +65,8 @@ cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecc
                           uint16_t* y, cudaStream_t s);
 cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                         const uint16_t* x, int batch, float* y, cudaStream_t s);
+cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
+                           const uint16_t* x, int batch, float* y, cudaStream_t s);
 cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s);
 cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats,
                                 cudaStream_t s);

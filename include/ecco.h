@@ -133,6 +133,7 @@ int ecco_decode(const ecco_tables* tables, const uint8_t* blocks, ecco_desc desc
 
 /* Fused decode + matrix-vector product ("Normalized memory requests for a
  * GEMM kernel", review page figure list): y[b][r] = sum_k W~[r][k] x[b][k],
+ * on CUDA cores for batch 1..4 and on the tcgen05 tensor cores for 5..16,
  * W~ the decoded rows x cols matrix whose blocks are stored row-major
  * (block (r, g) at index r * cols/128 + g), x_bf16 [batch][cols], y [batch][rows]
  * fp32.  cols % 128 == 0, 1 <= batch <= 16.  The decoded matrix is never
@@ -154,6 +155,12 @@ typedef struct {
 int ecco_decode_multi(const ecco_segment* segments, int n_segments, void* stream);
 int ecco_encode_multi(const ecco_segment* segments, int n_segments, ecco_stats* dev_stats,
                       void* stream);
+
+/* Number of bounded device-side waits (tensor-core decode+GEMV pipeline) that
+ * gave up since the library was loaded on the current device; 0 in normal
+ * operation.  A kernel whose wait gives up skips the rest of its work instead
+ * of hanging, so its outputs are incomplete.  Blocking (reads device memory). */
+int ecco_device_timeouts(unsigned int* out);
 
 const char* ecco_strerror(int code);
 int ecco_abi_version(void);

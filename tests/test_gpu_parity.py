@@ -364,3 +364,29 @@ def test_multi_segment_many_small_segments_cross_launches():
         np.testing.assert_array_equal(bits(y).reshape(-1, 128), oracle.decode(table_set(name), want, nthreads=4))
         tot += wst.n_groups
     assert ecco.read_stats(st)["n_groups"] == tot
+
+
+@pytest.mark.parametrize("batch", [5, 16])
+def test_tensor_core_gemv_one_hot_columns_are_exact(batch):
+    """Batch > 4 runs on tcgen05 tensor cores.  With x[b] one-hot at column c_b,
+    y[b] must be decoded column c_b bit for bit (one exact product per row)."""
+    blob = table_set("learned_w")
+    rows, cols = 700, 384
+    wb = inputs("t5", rows * cols // 128, seed=9)
+    blocks, _ = oracle.encode(blob, wb, nthreads=8)
+    Wd = oracle.decode(blob, blocks).reshape(rows, cols)
+    t = ecco.Tables(blob, DEV)
+    cs = [0, 17, 127, 128, 200, 255, 256, 383, 64, 300, 5, 130, 260, 99, 333, 1][:batch]
+    x = np.zeros((batch, cols), dtype=np.uint16)
+    for b, c in enumerate(cs):
+        x[b, c] = 0x3F80
+    y = ecco.decode_gemv(torch.from_numpy(blocks).to(DEV), t, rows, cols, to_dev_bf16(x)).cpu().numpy()
+    for b, c in enumerate(cs):
+        np.testing.assert_array_equal(y[b], (Wd[:, c].astype(np.uint32) << 16).view(np.float32))
+
+
+def test_no_device_wait_gave_up():
+    import ctypes
+    n = ctypes.c_uint(123)
+    assert _lib.load().ecco_device_timeouts(ctypes.byref(n)) == 0
+    assert n.value == 0
