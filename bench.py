@@ -4,9 +4,10 @@
 Default workload (`--workload kv`): one Llama-3-8B-shaped layer of KV cache,
 K and V each [8, 8, 4096, 128] bf16.  A step encodes the last 64 tokens of K
 and V (8,192 groups, written into the compressed cache) and decodes the whole
-compressed cache back to bf16 (524,288 blocks).  Other workloads:
-`c1` (256 x 1024 matrix, encode + decode), `mlp` (14336 x 4096 weight: encode,
-decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights,
+compressed cache back to bf16 (524,288 blocks); K and V go through one
+multi-segment launch each way (`encode_multi`, `decode_multi`).  Other
+workloads: `c1` (256 x 1024 matrix, encode + decode), `mlp` (14336 x 4096
+weight: encode, decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights,
 encode and decode of the whole set), `longctx` (32 layers x K,V x
 [1, 8, 131072, 128]: full streaming decode plus a one-token append per layer).
 
@@ -163,7 +164,9 @@ class KVWorkload(Workload):
                     V.view(self.rows, self.S, self.D)[:, self.S - self.T:].contiguous()]
         self.out = [torch.empty((self.n, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
         self.append = ecco.kv_append_desc(self.rows, self.T, self.S, self.S - self.T)
-        self.launches_per_step = 4
+        self.app = [ecco.Seg(self.tables[i], self.new[i], self.blocks[i], self.append) for i in range(2)]
+        self.dec = [ecco.Seg(self.tables[i], self.blocks[i], self.out[i]) for i in range(2)]
+        self.launches_per_step = 2
         self.dec_ms = []
 
     def bytes_decoded(self):
@@ -173,23 +176,22 @@ class KVWorkload(Workload):
         return 2 * self.rows * self.T * 256
 
     def step(self, record=False):
+        """K and V appended in one multi-segment launch, both caches decoded in one."""
         e = self.ecco
-        for i in range(2):
-            e.encode(self.new[i], self.tables[i], out=self.blocks[i], desc=self.append)
-        for i in range(2):
-            if record:
-                a, b = _events(self.torch)
-                a.record()
-            e.decode(self.blocks[i], self.tables[i], out=self.out[i])
-            if record:
-                b.record()
-                self.dec_ms.append((a, b))
+        e.encode_multi(self.app)
+        if record:
+            a, b = _events(self.torch)
+            a.record()
+        e.decode_multi(self.dec)
+        if record:
+            b.record()
+            self.dec_ms.append((a, b))
 
     def dominant(self):
         """(kernel name, algorithmic bytes per launch, launch ms list)."""
         self.torch.cuda.synchronize()
         ms = [a.elapsed_time(b) for a, b in self.dec_ms]
-        return "decode_kernel", self.n * (64 + 256), ms
+        return "decode_kernel", 2 * self.n * (64 + 256), ms
 
     # ---- end to end through the public API with host buffers
     def e2e_setup(self):
@@ -198,6 +200,7 @@ class KVWorkload(Workload):
         self.h_blocks = [b.cpu().pin_memory() for b in self.blocks]
         self.h_out = [torch.empty((self.n, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         self.d_new = [torch.empty_like(t) for t in self.new]
+        self.e2e_app = [self.ecco.Seg(self.tables[i], self.d_new[i], self.blocks[i], self.append) for i in range(2)]
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_new + self.h_blocks)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
 
@@ -206,8 +209,9 @@ class KVWorkload(Workload):
         for i in range(2):
             self.d_new[i].copy_(self.h_new[i], non_blocking=True)
             self.blocks[i].copy_(self.h_blocks[i], non_blocking=True)
-            e.encode(self.d_new[i], self.tables[i], out=self.blocks[i], desc=self.append)
-            e.decode(self.blocks[i], self.tables[i], out=self.out[i])
+        e.encode_multi(self.e2e_app)
+        e.decode_multi(self.dec)
+        for i in range(2):
             self.h_out[i].copy_(self.out[i], non_blocking=True)
 
     # ---- CPU oracle on a bounded sample of the same step
