@@ -25,8 +25,7 @@ constexpr int kWordStride = kDecThreads;  // word k of thread t at k * stride + 
 constexpr size_t kDecSmemLut = sizeof(((DevTables*)0)->lut);  // 65536
 constexpr size_t kDecSmemCt = sizeof(((DevTables*)0)->Ct);    // 4096
 constexpr size_t kDecSmemWords = 16 * kWordStride * 4;
-constexpr size_t kDecSmemSort = (size_t)kDecThreads * 16 + 260 * 4;  // block addresses by slot, bin counts
-constexpr size_t kDecSmem = kDecSmemLut + kDecSmemCt + kDecSmemWords + kDecSmemSort;
+constexpr size_t kDecSmem = kDecSmemLut + kDecSmemCt + kDecSmemWords;
 
 // WIDE: 32-byte stores (output 32-byte aligned), else 16-byte stores.
 template <bool WIDE>
@@ -69,10 +68,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kDecSmemLut);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kDecSmemLut + kDecSmemCt);
-    const uint8_t** s_src = reinterpret_cast<const uint8_t**>(smem + kDecSmemLut + kDecSmemCt + kDecSmemWords);
-    uint16_t** s_dst = reinterpret_cast<uint16_t**>(smem + kDecSmemLut + kDecSmemCt + kDecSmemWords +
-                                                    (size_t)kDecThreads * sizeof(void*));
-    uint32_t* s_bin = reinterpret_cast<uint32_t*>(s_dst + kDecThreads);
     const int tid = threadIdx.x;
     uint32_t* ws = s_w + tid;
 
@@ -90,53 +85,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         const float S_t = tb->S_t;
         __syncthreads();
 
-        // Rounds of kDecThreads consecutive groups.  Within a round the blocks
-        // are handed to threads sorted by codebook (header bits 8-15), so a
-        // warp's table lookups mostly hit one 256-entry table: lookups then
-        // conflict at most 2-way instead of landing in random banks.
+        // local group index within the segment; consecutive threads take
+        // consecutive groups, kDecThreads per round
         const int64_t gpr = S.d.groups_per_row;
         const int64_t stride_r = kDecThreads / gpr, stride_g = kDecThreads % gpr;
+        int64_t item = lo - S.begin + tid;
         const int64_t end = stop - S.begin;
-        int64_t base = lo - S.begin;
-        int64_t r = (base + tid) / gpr, g = (base + tid) - r * gpr;
-        for (; base < end; base += kDecThreads) {
-            const bool have = base + tid < end;
-            const uint8_t* my_src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * ECCO_BLOCK_BYTES;
-            uint16_t* my_dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * kG;
+        int64_t r = item / gpr, g = item - r * gpr;
+        for (; item < end; item += kDecThreads) {
+            const uint8_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * ECCO_BLOCK_BYTES;
+            uint16_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * kG;
             g += stride_g;
             r += stride_r;
             if (g >= gpr) {
                 g -= gpr;
                 r += 1;
             }
-            const uint32_t bin = have ? ((__ldg(reinterpret_cast<const uint32_t*>(my_src)) >> 8) & 255u) : 256u;
-            if (tid < 257) s_bin[tid] = 0u;
-            __syncthreads();
-            const uint32_t rank = atomicAdd(&s_bin[bin], 1u);
-            __syncthreads();
-            if (tid < 32) {  // exclusive scan of the 257 bin counts
-                uint32_t run = 0;
-                for (int c = 0; c < 9; ++c) {
-                    const int k = c * 32 + tid;
-                    const uint32_t v = k < 257 ? s_bin[k] : 0u;
-                    uint32_t inc = v;
-#pragma unroll
-                    for (int d = 1; d < 32; d <<= 1) {
-                        uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
-                        if (tid >= d) inc += t;
-                    }
-                    if (k < 257) s_bin[k] = run + inc - v;
-                    run += __shfl_sync(0xffffffffu, inc, 31);
-                }
-            }
-            __syncthreads();
-            const uint32_t slot = s_bin[bin] + rank;
-            s_src[slot] = my_src;
-            s_dst[slot] = my_dst;
-            __syncthreads();
-            if (tid >= (int)min((int64_t)kDecThreads, end - base)) continue;
-            const uint8_t* src = s_src[tid];
-            uint16_t* dst = s_dst[tid];
 
             uint4 q0 = ldg_nc_v4(src), q1 = ldg_nc_v4(src + 16), q2 = ldg_nc_v4(src + 32),
                   q3 = ldg_nc_v4(src + 48);
