@@ -23,6 +23,7 @@ GROUP = 128
 BLOCK_BYTES = 64
 
 __all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
+           "decode_attention", "attention_workspace_bytes",
            "new_stats", "read_stats", "flat_desc", "kv_append_desc", "EccoError", "Desc"]
 
 
@@ -150,6 +151,43 @@ def decode_gemv(blocks: torch.Tensor, tables: Tables, rows: int, cols: int, x: t
                                       ctypes.c_void_p(x.data_ptr()), batch,
                                       ctypes.c_void_p(out.data_ptr()), _stream(x.device))
     _lib.check(rc, "ecco_decode_gemv")
+    return out
+
+
+def attention_workspace_bytes(batch: int, kv_heads: int, group: int, seq_len: int) -> int:
+    return int(_lib.load().ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len))
+
+
+def decode_attention(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: Tables, v_tables: Tables,
+                     q: torch.Tensor, seq_len: int, scale: float, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode-phase attention over a compressed KV cache.
+
+    k_blocks / v_blocks: uint8 [B, Hkv, S_cap, 64]; q: bf16 [B, Hkv * G, 128].
+    Returns fp32 [B, Hkv * G, 128]: softmax over the first seq_len tokens of
+    scale * q . K~, applied to V~ (K~, V~ decoded inside the kernel)."""
+    _check_tensor(k_blocks, torch.uint8, "k_blocks", k_tables.device)
+    _check_tensor(v_blocks, torch.uint8, "v_blocks", v_tables.device)
+    _check_tensor(q, torch.bfloat16, "q", k_tables.device)
+    if k_blocks.dim() != 4 or k_blocks.shape[-1] != BLOCK_BYTES or v_blocks.shape != k_blocks.shape:
+        raise ValueError("k_blocks / v_blocks must be [B, Hkv, S_cap, 64] of the same shape")
+    B, H, s_cap, _ = k_blocks.shape
+    if q.dim() != 3 or q.shape[0] != B or q.shape[2] != GROUP or q.shape[1] % H:
+        raise ValueError("q must be [B, Hkv * G, 128]")
+    G = q.shape[1] // H
+    if out is None:
+        out = torch.empty((B, H * G, GROUP), dtype=torch.float32, device=q.device)
+    _check_tensor(out, torch.float32, "out", k_tables.device)
+    need = attention_workspace_bytes(B, H, G, seq_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check_tensor(workspace, torch.uint8, "workspace", k_tables.device)
+    rc = _lib.load().ecco_decode_attention(
+        k_tables.handle, v_tables.handle, ctypes.c_void_p(k_blocks.data_ptr()),
+        ctypes.c_void_p(v_blocks.data_ptr()), s_cap, B, H, G, int(seq_len), ctypes.c_void_p(q.data_ptr()),
+        float(scale), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel(), _stream(q.device))
+    _lib.check(rc, "ecco_decode_attention")
     return out
 
 

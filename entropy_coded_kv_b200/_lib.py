@@ -21,7 +21,8 @@ MAX_SEGMENTS = 256
 EXPORTED = [
     "ecco_tables_create", "ecco_tables_destroy", "ecco_select_encode", "ecco_decode",
     "ecco_decode_gemv", "ecco_decode_multi", "ecco_encode_multi", "ecco_strerror",
-    "ecco_abi_version", "ecco_device_timeouts",
+    "ecco_abi_version", "ecco_device_timeouts", "ecco_decode_attention",
+    "ecco_decode_attention_workspace_bytes",
 ]
 
 
@@ -67,9 +68,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_strerror.restype = ctypes.c_char_p
     L.ecco_abi_version.argtypes = []
     L.ecco_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    L.ecco_decode_attention_workspace_bytes.argtypes = [I, I, I, I]
+    L.ecco_decode_attention.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P,
+                                        ctypes.c_size_t, P]
     for fn in EXPORTED:
-        if fn != "ecco_strerror":
+        if fn not in ("ecco_strerror", "ecco_decode_attention_workspace_bytes"):
             getattr(L, fn).restype = I
+    L.ecco_decode_attention_workspace_bytes.restype = ctypes.c_size_t
     _lib = L
     return L
 

@@ -129,12 +129,39 @@ extern "C" int ecco_encode_multi(const ecco_segment* segs, int n, ecco_stats* st
     return status(launch_encode_multi(segs, n, stats, (cudaStream_t)stream));
 }
 
+extern "C" size_t ecco_decode_attention_workspace_bytes(int batch, int kv_heads, int group, int seq_len)
+{
+    if (batch < 1 || kv_heads < 1 || group < 1 || group > 8 || seq_len < 1) return 0;
+    return sizeof(float) * 130 * (size_t)batch * (size_t)kv_heads * (size_t)group *
+           (size_t)attention_splits(seq_len);
+}
+
+extern "C" int ecco_decode_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                                     const uint8_t* vblk, int64_t s_cap, int batch, int kv_heads,
+                                     int group, int seq_len, const uint16_t* q, float scale, float* out,
+                                     void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_tables(kt);
+    if (rc) return rc;
+    if ((rc = check_tables(vt))) return rc;
+    if (batch < 1 || kv_heads < 1 || group < 1 || group > 8 || seq_len < 1 || s_cap < seq_len)
+        return ECCO_ERR_ARG;
+    if ((int64_t)batch * kv_heads > 65535 || s_cap > ((int64_t)1 << 34)) return ECCO_ERR_ARG;
+    if (!kblk || !vblk || !q || !out || !ws) return ECCO_ERR_ARG;
+    if (ws_bytes < ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len)) return ECCO_ERR_ARG;
+    if (!aligned16(kblk) || !aligned16(vblk) || (reinterpret_cast<uintptr_t>(q) & 1u) ||
+        (reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 3u))
+        return ECCO_ERR_ALIGN;
+    return status(launch_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, scale,
+                                   out, static_cast<float*>(ws), (cudaStream_t)stream));
+}
+
 extern "C" const char* ecco_strerror(int code)
 {
     switch (code) {
         case ECCO_OK: return "ok";
         case ECCO_ERR_ARG: return "invalid argument";
-        case ECCO_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ECCO_ERR_ALIGN: return "pointer not aligned as required";
         case ECCO_ERR_TABLES: return "invalid table blob";
         case ECCO_ERR_CUDA: return "CUDA runtime error";
         case ECCO_ERR_DEVICE: return "current device is not the tables' device";

@@ -71,6 +71,12 @@ cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s)
 cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats,
                                 cudaStream_t s);
 
+// Attention over a compressed KV cache: splits of 512 tokens, then a merge.
+int attention_splits(int seq_len);
+cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                             const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
+                             const uint16_t* q, float scale, float* out, float* ws, cudaStream_t s);
+
 int device_sm_count();
 
 // ------------------------------------------------------------ device helpers

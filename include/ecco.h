@@ -51,7 +51,7 @@ extern "C" {
 
 #define ECCO_OK 0
 #define ECCO_ERR_ARG (-1)         /* null/negative/inconsistent argument */
-#define ECCO_ERR_ALIGN (-2)       /* pointer not 16-byte aligned */
+#define ECCO_ERR_ALIGN (-2)       /* pointer not aligned as the call requires */
 #define ECCO_ERR_TABLES (-3)      /* table blob invalid */
 #define ECCO_ERR_CUDA (-4)        /* CUDA runtime error (launch, copy, device) */
 #define ECCO_ERR_DEVICE (-5)      /* current device is not the tables' device */
@@ -155,6 +155,33 @@ typedef struct {
 int ecco_decode_multi(const ecco_segment* segments, int n_segments, void* stream);
 int ecco_encode_multi(const ecco_segment* segments, int n_segments, ecco_stats* dev_stats,
                       void* stream);
+
+/* Decode-phase attention read straight from a compressed KV cache (the
+ * memory-bound decode phase at long sequence lengths where the review page
+ * places Ecco's gains: "If this is right", Fig. 11 caption).  The K and V
+ * blocks are decoded inside the attention kernel; the bf16 cache is never
+ * materialised.  For batch b and query head j (KV head h = j / group):
+ *   out[b][j][:] = sum_s p_s V~[b][h][s][:],
+ *   p = softmax_s(scale * (q[b][j] . K~[b][h][s])),  0 <= s < seq_len,
+ * with K~, V~ the values ecco_decode would produce.
+ *   k_blocks, v_blocks  [batch][kv_heads][seq_capacity] blocks (64 B each; token s
+ *                       of head h at index (b * kv_heads + h) * seq_capacity + s),
+ *                       16-byte aligned; k_tables / v_tables decode them;
+ *   q_bf16              [batch][kv_heads * group][128] bf16, 2-byte aligned;
+ *   out                 [batch][kv_heads * group][128] fp32, 4-byte aligned;
+ *   workspace           caller-owned device scratch of at least
+ *                       ecco_decode_attention_workspace_bytes(...) bytes,
+ *                       4-byte aligned; no initial contents are needed and it
+ *                       holds per-split partial results afterwards.
+ * 1 <= group <= 8, 1 <= seq_len <= seq_capacity, batch, kv_heads >= 1.
+ * Two calls that share a workspace must be ordered (same stream).  Summation
+ * order is unspecified (fp32 accumulation, fp32 exp). */
+size_t ecco_decode_attention_workspace_bytes(int batch, int kv_heads, int group, int seq_len);
+int ecco_decode_attention(const ecco_tables* k_tables, const ecco_tables* v_tables,
+                          const uint8_t* k_blocks, const uint8_t* v_blocks, int64_t seq_capacity,
+                          int batch, int kv_heads, int group, int seq_len, const uint16_t* q_bf16,
+                          float scale, float* out, void* workspace, size_t workspace_bytes,
+                          void* stream);
 
 /* Number of bounded device-side waits (tensor-core decode+GEMV pipeline) that
  * gave up since the library was loaded on the current device; 0 in normal

@@ -18,7 +18,7 @@ def declared():
     for f in os.listdir(os.path.join(ROOT, "include")):
         if f.endswith(".h"):
             src = open(os.path.join(ROOT, "include", f)).read()
-            names |= set(re.findall(r"^\s*(?:int|const char\s*\*)\s+(ecco_\w+)\s*\(", src, re.M))
+            names |= set(re.findall(r"^\s*(?:int|size_t|const char\s*\*)\s+(ecco_\w+)\s*\(", src, re.M))
     return names
 
 
@@ -55,6 +55,13 @@ def test_argument_errors_need_no_gpu(lib):
     h = ctypes.c_void_p()
     assert lib.ecco_tables_create(None, 7952, ctypes.byref(h)) == _lib.ECCO_ERR_ARG
     assert lib.ecco_tables_create(b"x" * 10, 10, ctypes.byref(h)) == _lib.ECCO_ERR_TABLES
+    assert lib.ecco_decode_attention(None, None, None, None, 64, 1, 1, 1, 1, None, 1.0, None, None, 0,
+                                     None) == _lib.ECCO_ERR_ARG
+    # workspace: 130 floats (128 partial sums, max, sum) per query head and 512-token split
+    assert lib.ecco_decode_attention_workspace_bytes(2, 8, 4, 4096) == 4 * 130 * 2 * 8 * 4 * 8
+    assert lib.ecco_decode_attention_workspace_bytes(1, 1, 1, 513) == 4 * 130 * 2
+    assert lib.ecco_decode_attention_workspace_bytes(1, 1, 9, 10) == 0
+    assert lib.ecco_decode_attention_workspace_bytes(1, 1, 1, 0) == 0
     bad = bytearray(7952)
     assert lib.ecco_tables_create(bytes(bad), 7952, ctypes.byref(h)) == _lib.ECCO_ERR_TABLES
 
