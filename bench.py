@@ -9,7 +9,9 @@ multi-segment launch each way (`encode_multi`, `decode_multi`).  Other
 workloads: `c1` (256 x 1024 matrix, encode + decode), `mlp` (14336 x 4096
 weight: encode, decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights,
 encode and decode of the whole set), `longctx` (32 layers x K,V x
-[1, 8, 131072, 128]: full streaming decode plus a one-token append per layer).
+[1, 8, 131072, 128]: full streaming decode plus a one-token append per layer),
+`attn` (one-token append + fused decode+attention over the compressed cache of
+the `kv` layer, 32 query heads).
 
 Prints ONE JSON line (rank 0).  `value` is whole-job bf16 GB/s: bf16 bytes the
 step decodes plus bf16 bytes it encodes, over all ranks, per second of device
@@ -40,7 +42,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ecco", choices=["ecco", "reference"])
-    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx"])
+    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
@@ -557,8 +559,108 @@ class LongCtxWorkload(Workload):
                 "what": f"the per-step append (512 groups) + decode of {nb} blocks (1/{round(1 / frac)} of the cache)"}
 
 
+class AttnWorkload(Workload):
+    """One decode step of attention over a compressed KV cache: append the new
+    token's K and V, then attention of 32 query heads (group 4) over all 4096
+    tokens, the blocks decoded inside the attention kernel."""
+    name = "attn"
+    B, H, S, D, G = 8, 8, 4096, 128, 4
+
+    def __init__(self, dev, seed_offset=0):
+        import torch
+        import workloads as W
+        import entropy_coded_kv_b200 as ecco
+        from entropy_coded_kv_b200.calib import learn_tables
+        self.torch, self.ecco, self.dev = torch, ecco, dev
+        self.desc = ("decode-phase attention over a compressed Llama-3-8B-shaped layer KV cache: K, V "
+                     "[8, 8, 4096, 128] as 64-byte blocks, 32 query heads (group 4); a step appends one "
+                     "token's K and V (128 groups) and runs fused decode+attention over all 4096 tokens")
+        K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
+        Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
+        self.tables = [ecco.Tables(learn_tables(Kc, seed=0), dev), ecco.Tables(learn_tables(Vc, seed=0), dev)]
+        self.rows = self.B * self.H
+        self.n = self.rows * self.S
+        self.blocks = [ecco.encode(K, self.tables[0]).view(self.B, self.H, self.S, 64),
+                       ecco.encode(V, self.tables[1]).view(self.B, self.H, self.S, 64)]
+        self.new = [K.view(self.rows, self.S, self.D)[:, self.S - 1:].contiguous(),
+                    V.view(self.rows, self.S, self.D)[:, self.S - 1:].contiguous()]
+        self.append = ecco.kv_append_desc(self.rows, 1, self.S, self.S - 1)
+        self.app = [ecco.Seg(self.tables[i], self.new[i], self.blocks[i], self.append) for i in range(2)]
+        g = torch.Generator(device=dev).manual_seed(77 + seed_offset)
+        self.q = torch.randn(self.B, self.H * self.G, self.D, generator=g, device=dev).to(torch.bfloat16)
+        self.out = torch.empty(self.B, self.H * self.G, self.D, dtype=torch.float32, device=dev)
+        self.ws = torch.empty(ecco.attention_workspace_bytes(self.B, self.H, self.G, self.S), dtype=torch.uint8,
+                              device=dev)
+        self.scale = 1.0 / self.D ** 0.5
+        self.launches_per_step = 3  # append (one multi-segment launch), split kernel, merge kernel
+        self.api = "entropy_coded_kv_b200.encode_multi/decode_attention (C ABI) with pinned host buffers"
+        self.att_ms = []
+
+    def bytes_decoded(self):  # bf16 K and V bytes the attention kernel decodes (consumed on chip)
+        return 2 * self.n * 256
+
+    def bytes_encoded(self):
+        return 2 * self.rows * 256
+
+    def cpu_frac(self):
+        return 1.0 / 64
+
+    def _attend(self, q):
+        return self.ecco.decode_attention(self.blocks[0], self.blocks[1], self.tables[0], self.tables[1], q,
+                                          self.S, self.scale, out=self.out, workspace=self.ws)
+
+    def step(self, record=False):
+        self.ecco.encode_multi(self.app)
+        if record:
+            a, b = _events(self.torch)
+            a.record()
+        self._attend(self.q)
+        if record:
+            b.record()
+            self.att_ms.append((a, b))
+
+    def dominant(self):
+        """Algorithmic bytes: compressed K and V read once, q read, output written."""
+        self.torch.cuda.synchronize()
+        ms = [a.elapsed_time(b) for a, b in self.att_ms]
+        nbytes = 2 * self.n * 64 + self.q.numel() * 2 + self.out.numel() * 4
+        return "attn_split_kernel+attn_merge_kernel", nbytes, ms
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.h_new = [t.cpu().pin_memory() for t in self.new]
+        self.h_q = self.q.cpu().pin_memory()
+        self.h_out = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.d_new = [torch.empty_like(t) for t in self.new]
+        self.d_q = torch.empty_like(self.q)
+        self.e2e_app = [self.ecco.Seg(self.tables[i], self.d_new[i], self.blocks[i], self.append) for i in range(2)]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_new) + self.h_q.numel() * 2
+        self.d2h = self.h_out.numel() * 4
+
+    def e2e_step(self):
+        for i in range(2):
+            self.d_new[i].copy_(self.h_new[i], non_blocking=True)
+        self.d_q.copy_(self.h_q, non_blocking=True)
+        self.ecco.encode_multi(self.e2e_app)
+        self._attend(self.d_q)
+        self.h_out.copy_(self.out, non_blocking=True)
+
+    def cpu_sample(self, frac):
+        import workloads as W
+        pairs = max(1, int(self.rows * frac))
+        kb = [self.blocks[i].view(self.rows, self.S, 64)[:pairs].cpu().numpy() for i in range(2)]
+        qb = W.bf16_bits(self.q.view(self.rows, self.G, self.D)[:pairs])
+        xs = [W.bf16_bits(self.new[i][:pairs].reshape(-1, 128)) for i in range(2)]
+        blobs = [t.blob for t in self.tables]
+        return {"enc": [(blobs[i], xs[i]) for i in range(2)], "dec": [],
+                "attn": (blobs, kb, qb, self.S, self.scale),
+                "bytes": 2 * pairs * self.S * 256 + 2 * pairs * 256,
+                "what": f"append + attention for {pairs} of {self.rows} (batch, KV head) pairs "
+                        f"({2 * pairs * self.S} blocks decoded)"}
+
+
 WORKLOADS = {"kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload, "model": ModelWorkload,
-             "longctx": LongCtxWorkload}
+             "longctx": LongCtxWorkload, "attn": AttnWorkload}
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -569,6 +671,10 @@ def time_oracle(sample, nthreads):
         oracle.encode(blob, xb, nthreads=nthreads)
     for blob, bl in sample["dec"]:
         oracle.decode(blob, bl, nthreads=nthreads)
+    if "attn" in sample:
+        (kt, vt), (kb, vb), qb, S, scale = sample["attn"]
+        n = kb.shape[0]
+        oracle.attention(kt, vt, kb.reshape(n, 1, S, 64), vb.reshape(n, 1, S, 64), qb, S, scale)
     return time.perf_counter() - t0
 
 
@@ -681,7 +787,7 @@ def main():
         ems = float(et.item())
         e2e = {"value": round(units / (ems * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ems, 4),
                "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
-               "api": "entropy_coded_kv_b200.encode/decode (C ABI) with pinned host buffers"}
+               "api": getattr(wl, "api", "entropy_coded_kv_b200.encode/decode (C ABI) with pinned host buffers")}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

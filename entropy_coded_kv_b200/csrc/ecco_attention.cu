@@ -8,17 +8,23 @@
 // V blocks, so the bf16 cache is never written to or read from memory.
 //
 // For each (batch b, KV head h) the sequence is cut into splits of 512 tokens
-// (flash-decoding).  One CTA of 512 threads owns a split; thread t owns token
-// split * 512 + t:
-//   K pass  decode the token's K block and form the G query heads' scores
-//           q . k~ * scale on the fly (q broadcast from shared memory);
-//           outlier records correct the dot products by (new - old) * q.
-//   softmax CTA-wide max and exp per query head.
-//   V pass  decode the token's V block; every 32 dimensions the warp
-//           transposes its 32 tokens through shared memory so that each lane
-//           accumulates p . v~ for one dimension, then adds it to the CTA's
-//           [G][128] accumulator (shared-memory atomics); records add
-//           p * (new - old) to the same accumulator.
+// (flash-decoding).  One CTA of 512 threads owns a split; thread t decodes
+// token split * 512 + t, one Huffman walk per block (the serial part).  The
+// two contractions run on the tensor cores as warp-level mma.sync tiles (bf16
+// inputs, fp32 accumulation), fed from a per-warp staging tile that holds the
+// warp's 32 tokens x 32 dimensions at a time:
+//   K pass  S[head][token] += Q[head][dims] . K[token][dims]^T
+//           (m16n8k16: rows = query heads of the group, n = 8 tokens,
+//           k = 16 dimensions; B fragments by ldmatrix from the token rows);
+//   softmax CTA-wide max and sum per head; the score fragments stay in
+//           registers and become the A fragments of the next product;
+//   V pass  O[head][dims] += P[head][tokens] . V[tokens][dims]
+//           (n = 8 dimensions, k = 16 tokens; B fragments by ldmatrix.trans).
+//           P is split into bf16 hi + lo parts carried in rows 0-7 and 8-15
+//           of the A operand, so O = rows 0-7 + rows 8-15 keeps p to about
+//           2^-17 relative while V enters exactly.
+// Outlier records change single elements after the walk: their effect is
+// added as (new - old) * q on the score and p * (new - old) on the output.
 // Partial (max, sum, p.V) of every split go to a caller-owned workspace; a
 // second kernel merges the splits with the usual log-sum-exp rescaling.
 #include "ecco_block.cuh"
@@ -29,7 +35,9 @@ namespace {
 constexpr int kAtThreads = 512;
 constexpr int kAtWarps = kAtThreads / 32;
 constexpr int kAtStride = kAtThreads;
-constexpr int kStageRow = 20;  // words per staged token row (32 bf16 + pad: conflict-free)
+constexpr int kStageRow = 20;  // words per staged token row: 32 bf16 + 16 B pad (ldmatrix conflict-free)
+constexpr int kHeads = 8;      // rows 0-7 of an m16 tile: the query heads of one KV head
+constexpr int kQbRow = 136;    // bf16 per staged q row (padded: conflict-free fragment loads)
 
 struct AttnArgs {
     const DevTables* ktb;
@@ -43,16 +51,42 @@ struct AttnArgs {
     float* ws;  // [B][H*G][splits][130]: 128 partial p.V, then max, sum
 };
 
-template <int G>
-constexpr size_t attn_smem()
+// shared memory map (bytes)
+constexpr size_t kOffLut = 0;
+constexpr size_t kOffCt = kOffLut + 65536;
+constexpr size_t kOffWords = kOffCt + 4096;
+constexpr size_t kOffNib = kOffWords + (size_t)16 * kAtStride * 4;      // [chunk][thread] symbol nibbles
+constexpr size_t kOffStage = kOffNib + (size_t)16 * kAtStride * 4;
+constexpr size_t kOffX = kOffStage + (size_t)kAtWarps * 32 * kStageRow * 4;  // [warp][token][head] f32
+constexpr size_t kOffQf = kOffX + (size_t)kAtWarps * 32 * kHeads * 4;         // [head][128] f32
+constexpr size_t kOffQb = kOffQf + (size_t)kHeads * 128 * 4;                  // [head][kQbRow] bf16
+constexpr size_t kOffRed = kOffQb + (size_t)kHeads * kQbRow * 2;              // [2][warp][head] f32
+constexpr size_t kOffAcc = kOffRed + (size_t)2 * kAtWarps * kHeads * 4;       // [head][128] f32
+constexpr size_t kAttnSmem = kOffAcc + (size_t)kHeads * 128 * 4;
+static_assert(kOffQb % 16 == 0 && kOffRed % 16 == 0 && kOffAcc % 16 == 0, "alignment");
+
+__device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
 {
-    return 65536 + 4096                           // decode tables, centroids
-           + (size_t)16 * kAtStride * 4           // stream words
-           + (size_t)kAtWarps * 32 * kStageRow * 4  // per-warp V staging
-           + (size_t)G * 128 * 4                  // q
-           + (size_t)G * kAtThreads * 4           // scores / probabilities
-           + (size_t)kAtWarps * G * 4 * 2         // reductions
-           + (size_t)G * 128 * 4;                 // p.V accumulator
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t r[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t r[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
 }
 
 // Loads one block, returns its scale (0 for a null scale or a token past the end).
@@ -78,69 +112,97 @@ __device__ __forceinline__ float value_of(const ValuePlanes& vp, uint32_t sym)
     return __uint_as_float((((ow >> sh) & 0xffu) | (((oh >> sh) & 0xffu) << 8)) << 16);
 }
 
-// Calls f(i, new_value - old_value) for every outlier record of an unclipped
-// block whose value is final (the last record of an element wins).
+// Calls f(i, new_value - old_value) once per element that an outlier record of
+// an unclipped block replaces, with the element's last record (which wins).
 template <class F>
-__device__ __forceinline__ void for_records(const Stream& st, const uint32_t* ws, int stride, float s,
-                                            const ValuePlanes& vp, const uint32_t nib[16], F f)
+__device__ __forceinline__ void for_records(const Stream& st, const uint32_t* ws, const uint32_t* nb, float s,
+                                            const ValuePlanes& vp, const float* o_of_q, F f)
 {
-    if (s == 0.0f || st.room < 0) return;
+    if (s == 0.0f || st.room < kRecBits) return;
     const int n = min(kMaxRec, st.room / kRecBits);
     const int at0 = kBlockBits - st.room;
+    uint32_t seen0 = 0, seen1 = 0, seen2 = 0, seen3 = 0;  // elements already given by a later record
     for (int k = n - 1; k >= 0; --k) {
-        const uint32_t rec = read_record(ws, stride, at0 + k * kRecBits);
+        const uint32_t rec = read_record(ws, kAtStride, at0 + k * kRecBits);
         const int i = (int)(rec & 127u);
-        bool later = false;
-        for (int k2 = k + 1; k2 < n; ++k2)
-            later = later || ((int)(read_record(ws, stride, at0 + k2 * kRecBits) & 127u) == i);
-        if (later) continue;
-        const int qv = (int)(int8_t)(uint8_t)(rec >> 7);
-        const float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __fdiv_rn((float)qv, 127.0f))));
-        uint32_t word = nib[0];
-#pragma unroll
-        for (int c = 1; c < 16; ++c) word = ((i >> 3) == c) ? nib[c] : word;
-        const float ov = value_of(vp, (word >> (4 * (i & 7))) & 15u);
+        const uint32_t bit = 1u << (i & 31);
+        const uint32_t sw = (i < 64) ? ((i < 32) ? seen0 : seen1) : ((i < 96) ? seen2 : seen3);
+        if (sw & bit) continue;
+        if (i < 32) seen0 |= bit;
+        else if (i < 64) seen1 |= bit;
+        else if (i < 96) seen2 |= bit;
+        else seen3 |= bit;
+        const float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __ldg(o_of_q + (rec >> 7)))));
+        const float ov = value_of(vp, (nb[(i >> 3) * kAtStride] >> (4 * (i & 7))) & 15u);
         f(i, nv - ov);
     }
+}
+
+// Decodes the 32 symbols of quarter `qd` of this thread's block into its row
+// of the warp's staging tile; the symbols (nibbles) go to the thread's column
+// nb[k * kAtStride], k = chunk, for the record pass.
+__device__ __forceinline__ void decode_quarter(Stream& st, const uint8_t* lut, const uint32_t* ws,
+                                               const ValuePlanes& vp, uint32_t* row, uint32_t* nb, int qd)
+{
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t w[4];
+        nb[(qd * 4 + c4) * kAtStride] = chunk_values(st, lut, ws, kAtStride, vp, w);
+        *reinterpret_cast<uint4*>(row + 4 * c4) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)
+{
+    return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
 }
 
 template <int G>
 __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_constant__ AttnArgs A)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t* s_lut = smem;
-    float* s_Ct = reinterpret_cast<float*>(smem + 65536);
-    uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + 65536 + 4096);
-    uint32_t* s_stage = s_w + 16 * kAtStride;
-    float* s_q = reinterpret_cast<float*>(s_stage + kAtWarps * 32 * kStageRow);
-    float* s_p = s_q + G * 128;
-    float* s_red = s_p + G * kAtThreads;
-    float* s_acc = s_red + kAtWarps * G * 2;  // [G][128]: p.V of the split (shared atomics)
+    uint8_t* s_lut = smem + kOffLut;
+    float* s_Ct = reinterpret_cast<float*>(smem + kOffCt);
+    uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kOffWords);
+    float* s_x = reinterpret_cast<float*>(smem + kOffX);
+    float* s_qf = reinterpret_cast<float*>(smem + kOffQf);
+    uint16_t* s_qb = reinterpret_cast<uint16_t*>(smem + kOffQb);
+    float* s_red = reinterpret_cast<float*>(smem + kOffRed);
+    float* s_acc = reinterpret_cast<float*>(smem + kOffAcc);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;  // mma fragment coordinates
     const int split = blockIdx.x, bh = blockIdx.y;
     const int b = bh / A.H, h = bh - b * A.H;
     const int Hq = A.H * G;
-    const int s_tok = split * kAtThreads + tid;
-    const bool have = s_tok < A.S;
-    const int64_t blk = (int64_t)bh * A.s_cap + s_tok;
+    const int tok0 = split * kAtThreads + warp * 32;  // first token of this warp
+    const bool have = tok0 + lane < A.S;
+    const int64_t blk = (int64_t)bh * A.s_cap + tok0 + lane;
 
-    // q of the group's heads (fp32), corrections cleared
-    for (int i = tid; i < G * 128; i += kAtThreads) {
+    // q of the group's heads (rows >= G are zero), accumulator cleared
+    for (int i = tid; i < kHeads * 128; i += kAtThreads) {
         const int g = i >> 7, d = i & 127;
-        s_q[i] = bf16_bits_to_f32(A.q[((int64_t)b * Hq + h * G + g) * 128 + d]);
+        const uint16_t v = (g < G) ? A.q[((int64_t)b * Hq + h * G + g) * 128 + d] : (uint16_t)0;
+        s_qb[g * kQbRow + d] = v;
+        s_qf[i] = bf16_bits_to_f32(v);
         s_acc[i] = 0.0f;
     }
     stage_tables<kAtThreads>(A.ktb, s_lut, s_Ct, tid);
     __syncthreads();
 
     uint32_t* ws = s_w + tid;
-    uint32_t nib[16];
+    uint32_t* nb = reinterpret_cast<uint32_t*>(smem + kOffNib) + tid;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kOffStage) + warp * 32 * kStageRow;
+    uint32_t* row = stage + lane * kStageRow;
+    const uint32_t stage_sh = (uint32_t)__cvta_generic_to_shared(stage);
+    float* xw = s_x + warp * 32 * kHeads;
 
-    // ---------------- K pass: scores
-    float dot[G];
+    // ---------------- K pass: S = Q K^T for the warp's 32 tokens
+    float S[4][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) dot[g] = 0.0f;
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) S[nt][e] = 0.0f;
     {
         uint4 q0, q1, q2, q3;
         const float s = load_block(A.kblk + blk * ECCO_BLOCK_BYTES, have, q0, q1, q2, q3, A.ktb->S_t);
@@ -148,71 +210,100 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         const ValuePlanes vp = make_planes(s, s_Ct, (int)((q0.x >> 8) & 63u));
         const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
         Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
+        // qrow[j] = q[gid][2 (tig + j)], q[gid][2 (tig + j) + 1]
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(s_qb + gid * kQbRow) + tig;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            uint32_t w[4];
-            nib[c] = chunk_values(st, lut, ws, kAtStride, vp, w);
-            float v[8];
+        for (int qd = 0; qd < 4; ++qd) {
+            decode_quarter(st, lut, ws, vp, row, nb, qd);
+            __syncwarp();
+            const int j0 = qd * 16;  // dims 32 qd.. as bf16 pairs
+            const uint32_t a00 = qrow[j0], a02 = qrow[j0 + 4], a10 = qrow[j0 + 8], a12 = qrow[j0 + 12];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[2 * j] = __uint_as_float(w[j] << 16);
-                v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+            for (int nt = 0; nt < 4; ++nt) {
+                // matrices (lane >> 3): dims 0-7, 8-15, 16-23, 24-31 of tokens nt*8 + (lane & 7)
+                uint32_t bfr[4];
+                ldsm_x4(stage_sh + (uint32_t)(((nt * 8 + (lane & 7)) * kStageRow + (lane >> 3) * 4) * 4), bfr);
+                mma_bf16(S[nt], a00, 0u, a02, 0u, bfr[0], bfr[1]);
+                mma_bf16(S[nt], a10, 0u, a12, 0u, bfr[2], bfr[3]);
             }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float4 qa = *reinterpret_cast<const float4*>(s_q + g * 128 + 8 * c);
-                const float4 qb = *reinterpret_cast<const float4*>(s_q + g * 128 + 8 * c + 4);
-                dot[g] = fmaf(v[0], qa.x, dot[g]);
-                dot[g] = fmaf(v[1], qa.y, dot[g]);
-                dot[g] = fmaf(v[2], qa.z, dot[g]);
-                dot[g] = fmaf(v[3], qa.w, dot[g]);
-                dot[g] = fmaf(v[4], qb.x, dot[g]);
-                dot[g] = fmaf(v[5], qb.y, dot[g]);
-                dot[g] = fmaf(v[6], qb.z, dot[g]);
-                dot[g] = fmaf(v[7], qb.w, dot[g]);
-            }
+            __syncwarp();
         }
-        for_records(st, ws, kAtStride, s, vp, nib, [&](int i, float dv) {
+        // outlier records: score += (new - old) * q[g][i], exchanged through shared memory
+        float corr[kHeads];
 #pragma unroll
-            for (int g = 0; g < G; ++g) dot[g] = fmaf(dv, s_q[g * 128 + i], dot[g]);
+        for (int g = 0; g < kHeads; ++g) corr[g] = 0.0f;
+        bool any = false;
+        for_records(st, ws, nb, s, vp, A.ktb->o_of_q, [&](int i, float dv) {
+            any = true;
+#pragma unroll
+            for (int g = 0; g < G; ++g) corr[g] = fmaf(dv, s_qf[g * 128 + i], corr[g]);
         });
+        if (__any_sync(0xffffffffu, any)) {
+            *reinterpret_cast<float4*>(xw + lane * kHeads) = make_float4(corr[0], corr[1], corr[2], corr[3]);
+            *reinterpret_cast<float4*>(xw + lane * kHeads + 4) = make_float4(corr[4], corr[5], corr[6], corr[7]);
+            __syncwarp();
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                S[nt][0] += xw[(nt * 8 + 2 * tig) * kHeads + gid];
+                S[nt][1] += xw[(nt * 8 + 2 * tig + 1) * kHeads + gid];
+            }
+            __syncwarp();
+        }
     }
 
-    // ---------------- softmax over this split's tokens
-    float m[G], l[G];
+    // ---------------- softmax over this split's tokens (head = gid)
+    float mx = -INFINITY;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const float sc = have ? dot[g] * A.scale : -INFINITY;
-        float mx = sc;
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) s_red[warp * G + g] = mx;
-        dot[g] = sc;
-    }
+        for (int e = 0; e < 2; ++e) {
+            const bool ok = tok0 + nt * 8 + 2 * tig + e < A.S;
+            S[nt][e] = ok ? S[nt][e] * A.scale : -INFINITY;
+            mx = fmaxf(mx, S[nt][e]);
+        }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (tig == 0) s_red[warp * kHeads + gid] = mx;
     __syncthreads();
+    float M = -INFINITY;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float mx = -INFINITY;
-        for (int w = 0; w < kAtWarps; ++w) mx = fmaxf(mx, s_red[w * G + g]);
-        m[g] = mx;
-        const float p = have ? expf(dot[g] - mx) : 0.0f;
-        s_p[g * kAtThreads + tid] = p;
-        float sum = p;
+    for (int w = 0; w < kAtWarps; ++w) M = fmaxf(M, s_red[w * kHeads + gid]);
+    float sum = 0.0f;
 #pragma unroll
-        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) s_red[kAtWarps * G + warp * G + g] = sum;
-    }
-    __syncthreads();  // also: K tables no longer read
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float sum = 0.0f;
-        for (int w = 0; w < kAtWarps; ++w) sum += s_red[kAtWarps * G + w * G + g];
-        l[g] = sum;
-    }
+        for (int e = 0; e < 2; ++e) {
+            const float p = expf(S[nt][e] - M);  // exp(-inf) = 0 past the end
+            S[nt][e] = p;
+            sum += p;
+            xw[(nt * 8 + 2 * tig + e) * kHeads + gid] = p;  // p by token, for the V records
+        }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    if (tig == 0) s_red[kAtWarps * kHeads + warp * kHeads + gid] = sum;
+    __syncthreads();  // also: the K tables are no longer read
+    float L = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kAtWarps; ++w) L += s_red[kAtWarps * kHeads + w * kHeads + gid];
     stage_tables<kAtThreads>(A.vtb, s_lut, s_Ct, tid);
+
+    // A fragments of P, k-step ks = tokens 16 ks + (0..15):
+    // a0 / a2 (rows 0-7) = bf16(p), a1 / a3 (rows 8-15) = bf16(p - bf16(p))
+    uint32_t pa[2][4];
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const float p0 = S[2 * ks + half][0], p1 = S[2 * ks + half][1];
+            const uint32_t hi = pack2_bf16(p0, p1);
+            const float r0 = p0 - __uint_as_float(hi << 16), r1 = p1 - __uint_as_float(hi & 0xffff0000u);
+            pa[ks][2 * half] = hi;
+            pa[ks][2 * half + 1] = pack2_bf16(r0, r1);
+        }
+    }
     __syncthreads();
 
-    // ---------------- V pass
+    // ---------------- V pass: O = P V
     {
         uint4 q0, q1, q2, q3;
         const float s = load_block(A.vblk + blk * ECCO_BLOCK_BYTES, have, q0, q1, q2, q3, A.vtb->S_t);
@@ -220,43 +311,30 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         const ValuePlanes vp = make_planes(s, s_Ct, (int)((q0.x >> 8) & 63u));
         const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
         Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
-        uint32_t* stage = s_stage + warp * 32 * kStageRow;
-        const float* pw = s_p + warp * 32;  // probabilities of this warp's 32 tokens
 #pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t w[4];
-                nib[grp * 4 + c4] = chunk_values(st, lut, ws, kAtStride, vp, w);
-                *reinterpret_cast<uint4*>(stage + lane * kStageRow + 4 * c4) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+        for (int qd = 0; qd < 4; ++qd) {
+            decode_quarter(st, lut, ws, vp, row, nb, qd);
             __syncwarp();
-            // lane = dimension 32 * grp + lane; the warp's 32 tokens in turn
-            const uint16_t* col = reinterpret_cast<const uint16_t*>(stage) + lane;
-            float acc[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-#pragma unroll 2
-            for (int t = 0; t < 32; t += 4) {
-                float v[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) v[k] = bf16_bits_to_f32(col[(t + k) * 2 * kStageRow]);
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float4 p4 = *reinterpret_cast<const float4*>(pw + g * kAtThreads + t);
-                    acc[g] = fmaf(p4.x, v[0], acc[g]);
-                    acc[g] = fmaf(p4.y, v[1], acc[g]);
-                    acc[g] = fmaf(p4.z, v[2], acc[g]);
-                    acc[g] = fmaf(p4.w, v[3], acc[g]);
+            for (int nd = 0; nd < 4; ++nd) {
+                // matrices (lane >> 3): tokens 0-7, 8-15, 16-23, 24-31 of dims nd*8..; lane l addresses token l
+                uint32_t bfr[4];
+                ldsm_x4_t(stage_sh + (uint32_t)((lane * kStageRow + nd * 4) * 4), bfr);
+                float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma_bf16(o, pa[0][0], pa[0][1], pa[0][2], pa[0][3], bfr[0], bfr[1]);
+                mma_bf16(o, pa[1][0], pa[1][1], pa[1][2], pa[1][3], bfr[2], bfr[3]);
+                if (gid < G) {
+                    const int d = qd * 32 + nd * 8 + 2 * tig;
+                    atomicAdd(&s_acc[gid * 128 + d], o[0] + o[2]);
+                    atomicAdd(&s_acc[gid * 128 + d + 1], o[1] + o[3]);
                 }
             }
-#pragma unroll
-            for (int g = 0; g < G; ++g) atomicAdd(&s_acc[g * 128 + grp * 32 + lane], acc[g]);
             __syncwarp();
         }
-        for_records(st, ws, kAtStride, s, vp, nib, [&](int i, float dv) {
+        const float* pt = xw + lane * kHeads;  // this token's p per head
+        for_records(st, ws, nb, s, vp, A.vtb->o_of_q, [&](int i, float dv) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) atomicAdd(&s_acc[g * 128 + i], s_p[g * kAtThreads + tid] * dv);
+            for (int g = 0; g < G; ++g) atomicAdd(&s_acc[g * 128 + i], pt[g] * dv);
         });
     }
     __syncthreads();
@@ -267,12 +345,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         const int g = i >> 7, d = i & 127;
         out[((int64_t)g * A.splits + split) * 130 + d] = s_acc[i];
     }
-    if (tid == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            out[((int64_t)g * A.splits + split) * 130 + 128] = m[g];
-            out[((int64_t)g * A.splits + split) * 130 + 129] = l[g];
-        }
+    if (warp == 0 && tig == 0 && gid < G) {
+        out[((int64_t)gid * A.splits + split) * 130 + 128] = M;
+        out[((int64_t)gid * A.splits + split) * 130 + 129] = L;
     }
 }
 
@@ -301,12 +376,12 @@ cudaError_t run_attn(const AttnArgs& A, int B, cudaStream_t s, float* out)
     cudaGetDevice(&dev);
     if (configured != dev) {
         cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)attn_smem<G>());
+                                             (int)kAttnSmem);
         if (e != cudaSuccess) return e;
         configured = dev;
     }
     dim3 grid((unsigned)A.splits, (unsigned)(B * A.H));
-    attn_split_kernel<G><<<grid, kAtThreads, attn_smem<G>(), s>>>(A);
+    attn_split_kernel<G><<<grid, kAtThreads, kAttnSmem, s>>>(A);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_merge_kernel<<<B * A.H * G, 128, 0, s>>>(A.ws, A.splits, out);

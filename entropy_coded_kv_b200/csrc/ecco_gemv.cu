@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                 for (int k2 = k + 1; k2 < n; ++k2)
                     later = later || ((int)(read_record(ws, kGvStride, at0 + k2 * kRecBits) & 127u) == i);
                 if (later) continue;
-                int qv = (int)(int8_t)(uint8_t)(rec >> 7);
-                float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __fdiv_rn((float)qv, 127.0f))));
+                float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __ldg(&tb->o_of_q[rec >> 7]))));
                 uint32_t osym = (nibs[(i >> 3) * kGvThreads] >> (4 * (i & 7))) & 15u;
                 uint32_t ow = (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);
                 uint32_t oh = (osym < 8) ? ((osym < 4) ? vp.hi[0] : vp.hi[1]) : ((osym < 12) ? vp.hi[2] : vp.hi[3]);

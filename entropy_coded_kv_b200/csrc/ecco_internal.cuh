@@ -46,6 +46,7 @@ struct DevTables {
     float s_of_code[256];           // S_t * fp8(code); 0 for zero and NaN codes
     float inv_of_code[256];         // 1 / s_of_code (0 where s is 0)
     uint8_t code_of_mag[32768];     // E4M3(|x| / S_t), saturating, for every bf16 magnitude |x|
+    float o_of_q[256];              // outlier record value q / 127 (IEEE divide) for each 8-bit code of q
 };
 
 }  // namespace ecco

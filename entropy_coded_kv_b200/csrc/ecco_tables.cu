@@ -125,6 +125,7 @@ __global__ void scale_tables_kernel(DevTables* t)
         }
         t->s_of_code[i] = s;
         t->inv_of_code[i] = inv;
+        t->o_of_q[i] = __fdiv_rn((float)(int8_t)(uint8_t)i, 127.0f);
     }
 }
 
