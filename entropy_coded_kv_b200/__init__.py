@@ -23,7 +23,7 @@ GROUP = 128
 BLOCK_BYTES = 64
 
 __all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
-           "decode_attention", "attention_workspace_bytes",
+           "decode_attention", "attention_workspace_bytes", "decode_attention_static",
            "new_stats", "read_stats", "flat_desc", "kv_append_desc", "EccoError", "Desc"]
 
 
@@ -188,6 +188,32 @@ def decode_attention(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: T
         float(scale), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel(), _stream(q.device))
     _lib.check(rc, "ecco_decode_attention")
+    return out
+
+
+def decode_attention_static(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: Tables, v_tables: Tables,
+                            q: torch.Tensor, seq_len: int, scale: float,
+                            out: torch.Tensor | None = None) -> torch.Tensor:
+    """decode_attention with the library's static device workspace (no
+    workspace argument, nothing allocated by the call when `out` is given).
+    Calls that can overlap on one device race on that workspace."""
+    _check_tensor(k_blocks, torch.uint8, "k_blocks", k_tables.device)
+    _check_tensor(v_blocks, torch.uint8, "v_blocks", v_tables.device)
+    _check_tensor(q, torch.bfloat16, "q", k_tables.device)
+    if k_blocks.dim() != 4 or k_blocks.shape[-1] != BLOCK_BYTES or v_blocks.shape != k_blocks.shape:
+        raise ValueError("k_blocks / v_blocks must be [B, Hkv, S_cap, 64] of the same shape")
+    B, H, s_cap, _ = k_blocks.shape
+    if q.dim() != 3 or q.shape[0] != B or q.shape[2] != GROUP or q.shape[1] % H:
+        raise ValueError("q must be [B, Hkv * G, 128]")
+    G = q.shape[1] // H
+    if out is None:
+        out = torch.empty((B, H * G, GROUP), dtype=torch.float32, device=q.device)
+    _check_tensor(out, torch.float32, "out", k_tables.device)
+    rc = _lib.load().ecco_decode_attention_static(
+        k_tables.handle, v_tables.handle, ctypes.c_void_p(k_blocks.data_ptr()),
+        ctypes.c_void_p(v_blocks.data_ptr()), s_cap, B, H, G, int(seq_len), ctypes.c_void_p(q.data_ptr()),
+        float(scale), ctypes.c_void_p(out.data_ptr()), _stream(q.device))
+    _lib.check(rc, "ecco_decode_attention_static")
     return out
 
 

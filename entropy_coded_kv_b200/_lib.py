@@ -15,6 +15,8 @@ ECCO_ERR_TABLES = -3
 ECCO_ERR_CUDA = -4
 ECCO_ERR_DEVICE = -5
 ECCO_ERR_UNSUPPORTED = -6
+ECCO_ERR_WORKSPACE = -7
+ATTENTION_STATIC_WS_BYTES = 4 << 20
 TABLES_BYTES = 7952
 MAX_SEGMENTS = 256
 
@@ -22,7 +24,7 @@ EXPORTED = [
     "ecco_tables_create", "ecco_tables_destroy", "ecco_select_encode", "ecco_decode",
     "ecco_decode_gemv", "ecco_decode_multi", "ecco_encode_multi", "ecco_strerror",
     "ecco_abi_version", "ecco_device_timeouts", "ecco_decode_attention",
-    "ecco_decode_attention_workspace_bytes",
+    "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static",
 ]
 
 
@@ -69,6 +71,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_abi_version.argtypes = []
     L.ecco_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     L.ecco_decode_attention_workspace_bytes.argtypes = [I, I, I, I]
+    L.ecco_decode_attention_static.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P]
     L.ecco_decode_attention.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P,
                                         ctypes.c_size_t, P]
     for fn in EXPORTED:

@@ -166,6 +166,7 @@ extern "C" const char* ecco_strerror(int code)
         case ECCO_ERR_CUDA: return "CUDA runtime error";
         case ECCO_ERR_DEVICE: return "current device is not the tables' device";
         case ECCO_ERR_UNSUPPORTED: return "device is not sm_100";
+        case ECCO_ERR_WORKSPACE: return "request needs more than the static attention workspace";
         default: return "unknown error";
     }
 }

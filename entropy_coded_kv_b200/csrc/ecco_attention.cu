@@ -27,6 +27,8 @@
 // added as (new - old) * q on the score and p * (new - old) on the output.
 // Partial (max, sum, p.V) of every split go to a caller-owned workspace; a
 // second kernel merges the splits with the usual log-sum-exp rescaling.
+#include <atomic>
+
 #include "ecco_block.cuh"
 
 namespace ecco {
@@ -411,3 +413,36 @@ cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const
 }
 
 }  // namespace ecco
+
+// ------------------------------------------------ static workspace variant
+// ecco_decode_attention_static: the split partials go to this file-scope
+// device array instead of a caller workspace, for callers that cannot allocate
+// device memory on the attention path (a plain-C host loop without a caching
+// allocator; code that must not call cudaMalloc, which can synchronize the
+// device and fail under memory pressure).  Nothing in it needs to start at
+// zero.  Calls that overlap on one device race on it.
+static __device__ __align__(256) float g_attn_static_ws[ECCO_ATTENTION_STATIC_WS_BYTES / sizeof(float)];
+
+static constexpr int kMaxDevices = 64;
+static std::atomic<void*> g_static_ws_addr[kMaxDevices];  // per device, looked up once with that device current
+
+extern "C" int ecco_decode_attention_static(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                                            const uint8_t* vblk, int64_t s_cap, int batch, int kv_heads,
+                                            int group, int seq_len, const uint16_t* q, float scale, float* out,
+                                            void* stream)
+{
+    const size_t need = ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len);
+    if (need == 0 || !kt || !vt) return ECCO_ERR_ARG;
+    if (need > (size_t)ECCO_ATTENTION_STATIC_WS_BYTES) return ECCO_ERR_WORKSPACE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ECCO_ERR_CUDA;
+    if (dev != kt->device || dev != vt->device) return ECCO_ERR_DEVICE;
+    if (dev < 0 || dev >= kMaxDevices) return ECCO_ERR_UNSUPPORTED;
+    void* ws = g_static_ws_addr[dev].load(std::memory_order_acquire);
+    if (!ws) {
+        if (cudaGetSymbolAddress(&ws, g_attn_static_ws) != cudaSuccess || !ws) return ECCO_ERR_CUDA;
+        g_static_ws_addr[dev].store(ws, std::memory_order_release);
+    }
+    return ecco_decode_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, scale, out, ws,
+                                 (size_t)ECCO_ATTENTION_STATIC_WS_BYTES, stream);
+}

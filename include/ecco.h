@@ -183,6 +183,31 @@ int ecco_decode_attention(const ecco_tables* k_tables, const ecco_tables* v_tabl
                           float scale, float* out, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* ecco_decode_attention with its workspace in static device memory: a
+ * file-scope __device__ array of ECCO_ATTENTION_STATIC_WS_BYTES per device
+ * inside the library, so the call allocates nothing and takes no workspace
+ * argument.  The pages have no counterpart to this entry point; it exists for
+ * callers that cannot allocate device memory where they run attention: a
+ * plain-C host loop has no caching allocator to draw a workspace from, and
+ * cudaMalloc can synchronize the device and fail under memory pressure.
+ *   - Requests whose workspace (ecco_decode_attention_workspace_bytes) exceeds
+ *     ECCO_ATTENTION_STATIC_WS_BYTES return ECCO_ERR_WORKSPACE and enqueue
+ *     nothing; other arguments and errors are those of ecco_decode_attention.
+ *   - Nothing in the workspace needs to start at zero: every split writes all
+ *     of its partial results before the merge reads them.
+ *   - The first call on each device looks up the workspace's address with that
+ *     device current (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - All calls on one device share the workspace: calls that can overlap (on
+ *     different streams, or from several host threads without ordering) race
+ *     on it and corrupt each other's results.  Order them on one stream. */
+#define ECCO_ATTENTION_STATIC_WS_BYTES (4u << 20)
+#define ECCO_ERR_WORKSPACE (-7) /* request needs more than the static workspace */
+int ecco_decode_attention_static(const ecco_tables* k_tables, const ecco_tables* v_tables,
+                                 const uint8_t* k_blocks, const uint8_t* v_blocks, int64_t seq_capacity,
+                                 int batch, int kv_heads, int group, int seq_len, const uint16_t* q_bf16,
+                                 float scale, float* out, void* stream);
+
 /* Number of bounded device-side waits (tensor-core decode+GEMV pipeline) that
  * gave up since the library was loaded on the current device; 0 in normal
  * operation.  A kernel whose wait gives up skips the rest of its work instead
