@@ -114,10 +114,14 @@ def lib():
             L.or_canonical_codes.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
             L.or_encode_group_ex.restype = None
             L.or_encode_group_ex.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int]
+            L.or_encode_group_sel.restype = None
+            L.or_encode_group_sel.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
             L.or_decode_block.restype = ctypes.c_int
             L.or_decode_block.argtypes = [P, P, P]
             L.or_encode.restype = None
             L.or_encode.argtypes = [P, P, I64, P, P, ctypes.c_int, ctypes.c_int]
+            L.or_encode_sel.restype = None
+            L.or_encode_sel.argtypes = [P, P, I64, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
             L.or_decode.restype = None
             L.or_decode.argtypes = [P, P, I64, P, ctypes.c_int]
             L.or_gemv.restype = None
@@ -182,14 +186,20 @@ def canonical_codes(tables, p: int, h: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- codec
-def encode_group(tables, x, force_p: int = -1, force_h: int = -1):
-    """One group: returns (block bytes [64] uint8, GroupInfo)."""
+SELECT_MINMAX = 0   # R8: min/max squared error (the method)
+SELECT_MSE = 1      # R23: full squared error, pairwise fp32 sum
+
+
+def encode_group(tables, x, force_p: int = -1, force_h: int = -1, select: int = SELECT_MINMAX,
+                 npat: int = NPAT):
+    """One group: returns (block bytes [64] uint8, GroupInfo).  `select` and
+    `npat` (patterns searched, R24) pick the selection variant."""
     b = _blob(tables)
     xb = _bits(x).reshape(-1)
-    assert xb.size == G
+    assert xb.size == G and 1 <= npat <= NPAT
     blk = np.zeros(BLOCK_BYTES, dtype=np.uint8)
     info = GroupInfo()
-    lib().or_encode_group_ex(_ptr(b), _ptr(xb), _ptr(blk), ctypes.byref(info), force_p, force_h)
+    lib().or_encode_group_sel(_ptr(b), _ptr(xb), _ptr(blk), ctypes.byref(info), select, npat, force_p, force_h)
     return blk, info
 
 
@@ -202,15 +212,19 @@ def decode_block(tables, blk) -> tuple[np.ndarray, int]:
     return y, int(k)
 
 
-def encode(tables, x, with_mse: bool = False, nthreads: int = 1):
-    """x: [..., 128*k] bf16 bits, contiguous groups.  Returns (blocks [n,64], Stats)."""
+def encode(tables, x, with_mse: bool = False, nthreads: int = 1, select: int = SELECT_MINMAX,
+           npat: int = NPAT):
+    """x: [..., 128*k] bf16 bits, contiguous groups.  Returns (blocks [n,64], Stats).
+    With with_mse, Stats.mse_minmax is the fp64 squared error of the chosen
+    patterns (whatever `select`), mse_full that of the fp64-best of all 64."""
     b = _blob(tables)
     xb = _bits(x).reshape(-1)
-    assert xb.size % G == 0
+    assert xb.size % G == 0 and 1 <= npat <= NPAT
     n = xb.size // G
     blocks = np.zeros((n, BLOCK_BYTES), dtype=np.uint8)
     st = Stats()
-    lib().or_encode(_ptr(b), _ptr(xb), n, _ptr(blocks), ctypes.byref(st), int(with_mse), nthreads)
+    lib().or_encode_sel(_ptr(b), _ptr(xb), n, _ptr(blocks), ctypes.byref(st), int(with_mse), nthreads,
+                        select, npat)
     return blocks, st
 
 

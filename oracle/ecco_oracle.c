@@ -49,6 +49,15 @@
  *   R18 scale codes 0x00, 0x80 (zero) and 0x7f, 0xff (NaN) decode to 128 x +0;
  *       records are applied in order (last wins).
  *   R21 a NaN or +-Inf input element is encoded as +0.0 and counted.
+ *   R23 full-MSE selection (the comparison the referee report asks for, major
+ *       comment 2; "What carries the argument" calls min/max a way of avoiding
+ *       full MSE): e_p = pairwise sum over the 128 element slots, in index
+ *       order, of d_i * d_i with d_i = u_i - C[p][sym_p(u_i)]; slot m adds +0.
+ *       Pairwise = a perfect binary tree (slots 0..63 + slots 64..127, each
+ *       half the same way).  Every op one fp32 rounding; first p with the least e_p.
+ *   R24 the compressor's pattern count (free parameters: "Shared k-means
+ *       patterns used in the compressor = 16, reduced from 64"): selection
+ *       searches patterns 0..npat-1 only; the block format is unchanged.
  *
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC -pthread.
  * Shares no source with the CUDA library.
@@ -288,9 +297,32 @@ static double pattern_mse(const or_tables* t, int p, const float* u, int m)
     return acc;
 }
 
-/* force_p / force_h < 0: the method's own choice; >= 0: forced (tests only). */
-void or_encode_group_ex(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
-                        or_group_info* info, int force_p, int force_h)
+/* R23: pairwise (perfect binary tree) fp32 sum of n = 2^k values. */
+static float pairwise_sum(const float* v, int n)
+{
+    if (n == 1) return v[0];
+    float a = pairwise_sum(v, n / 2);
+    float b = pairwise_sum(v + n / 2, n / 2);
+    return a + b;
+}
+
+/* R23: full squared error of the normalised group under pattern p. */
+static float pattern_sq_error(const or_tables* t, int p, const float* u, int m)
+{
+    float d2[OR_G];
+    for (int i = 0; i < OR_G; ++i) {
+        if (i == m) { d2[i] = 0.0f; continue; }
+        float d = u[i] - t->C[p][quantise(t, p, u[i])];
+        d2[i] = d * d;
+    }
+    return pairwise_sum(d2, OR_G);
+}
+
+/* select: 0 = min/max fitness (R8), 1 = full squared error (R23); npat = number
+ * of patterns the selection searches (R24, 1..64).  force_p / force_h < 0: the
+ * method's own choice; >= 0: forced (tests only). */
+void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
+                         or_group_info* info, int select, int npat, int force_p, int force_h)
 {
     or_group_info gi;
     memset(&gi, 0, sizeof gi);
@@ -342,12 +374,17 @@ void or_encode_group_ex(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
     gi.umin = umin;
     gi.umax = umax;
     int p = 0;
-    for (int q = 0; q < OR_NPAT; ++q) {
-        float d0 = umin - t->C[q][0];
-        float d1 = umax - t->C[q][OR_NCENT - 1];
-        float sq0 = d0 * d0;
-        float sq1 = d1 * d1;
-        float e = sq0 + sq1;
+    for (int q = 0; q < npat; ++q) {
+        float e;
+        if (select == 0) {
+            float d0 = umin - t->C[q][0];
+            float d1 = umax - t->C[q][OR_NCENT - 1];
+            float sq0 = d0 * d0;
+            float sq1 = d1 * d1;
+            e = sq0 + sq1;
+        } else {
+            e = pattern_sq_error(t, q, u, m);
+        }
         gi.e[q] = e;
         if (e < gi.e[p]) p = q;
     }
@@ -416,6 +453,12 @@ void or_encode_group_ex(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
         gi.n_rec = n;
     }
     if (info) *info = gi;
+}
+
+void or_encode_group_ex(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
+                        or_group_info* info, int force_p, int force_h)
+{
+    or_encode_group_sel(t, x_in, blk, info, 0, OR_NPAT, force_p, force_h);
 }
 
 void or_encode_group(const or_tables* t, const uint16_t* x, uint8_t* blk, or_group_info* info)
@@ -488,6 +531,7 @@ typedef struct {
     uint16_t* y;
     int64_t lo, hi;
     int with_mse;
+    int select, npat;
     or_stats st;
 } or_job;
 
@@ -496,7 +540,8 @@ static void* encode_worker(void* arg)
     or_job* j = (or_job*)arg;
     or_group_info gi;
     for (int64_t g = j->lo; g < j->hi; ++g) {
-        or_encode_group(j->t, j->x + g * OR_G, j->blocks + g * OR_BLOCK_BYTES, &gi);
+        or_encode_group_sel(j->t, j->x + g * OR_G, j->blocks + g * OR_BLOCK_BYTES, &gi, j->select, j->npat,
+                            -1, -1);
         j->st.n_groups += 1;
         j->st.n_nonfinite += (uint64_t)gi.nonfinite;
         if (gi.zero) { j->st.n_zero += 1; continue; }
@@ -566,8 +611,8 @@ static void run_jobs(void* (*fn)(void*), or_job* base, int64_t n, int nthreads, 
 }
 
 /* x: n_groups * 128 bf16, contiguous; blocks: n_groups * 64 bytes. */
-void or_encode(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
-               or_stats* stats, int with_mse, int nthreads)
+void or_encode_sel(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
+                   or_stats* stats, int with_mse, int nthreads, int select, int npat)
 {
     or_job base;
     memset(&base, 0, sizeof base);
@@ -575,7 +620,15 @@ void or_encode(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t*
     base.x = x;
     base.blocks = blocks;
     base.with_mse = with_mse;
+    base.select = select;
+    base.npat = npat;
     run_jobs(encode_worker, &base, n_groups, nthreads, stats);
+}
+
+void or_encode(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
+               or_stats* stats, int with_mse, int nthreads)
+{
+    or_encode_sel(t, x, n_groups, blocks, stats, with_mse, nthreads, 0, OR_NPAT);
 }
 
 void or_decode(const or_tables* t, const uint8_t* blocks, int64_t n_blocks, uint16_t* y,
