@@ -11,7 +11,9 @@ weight: encode, decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers
 encode and decode of the whole set), `longctx` (32 layers x K,V x
 [1, 8, 131072, 128]: full streaming decode plus a one-token append per layer),
 `attn` (one-token append + fused decode+attention over the compressed cache of
-the `kv` layer, 32 query heads).
+the `kv` layer, 32 query heads), `select` (encode of the `kv` layer with
+full-MSE pattern selection, plus a quality study of min/max vs full-MSE
+selection with 64 and 16 patterns).
 
 Prints ONE JSON line (rank 0).  `value` is whole-job bf16 GB/s: bf16 bytes the
 step decodes plus bf16 bytes it encodes, over all ranks, per second of device
@@ -42,7 +44,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ecco", choices=["ecco", "reference"])
-    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn"])
+    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
@@ -659,8 +661,112 @@ class AttnWorkload(Workload):
                         f"({2 * pairs * self.S} blocks decoded)"}
 
 
+class SelectWorkload(Workload):
+    """Pattern-selection study on the KV cache: a step encodes K and V of the
+    [8, 8, 4096, 128] layer with full-MSE pattern selection (64 patterns);
+    setup also times and scores min/max and the 16-pattern variants."""
+    name = "select"
+    B, H, S, D = 8, 8, 4096, 128
+
+    def __init__(self, dev, seed_offset=0):
+        import torch
+        import workloads as W
+        import entropy_coded_kv_b200 as ecco
+        from entropy_coded_kv_b200 import _lib
+        from entropy_coded_kv_b200.calib import learn_tables
+        self.torch, self.ecco, self.dev, self._lib = torch, ecco, dev, _lib
+        self.desc = ("KV cache [8, 8, 4096, 128] K and V: encode with full-MSE pattern selection over 64 "
+                     "patterns (524,288 groups); quality of min/max vs full-MSE selection, 64 and 16 patterns")
+        K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
+        Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
+        self.x = [K, V]
+        self.n = K.numel() // 128
+        self.tabs = {64: [ecco.Tables(learn_tables(c, seed=0), dev) for c in (Kc, Vc)],
+                     16: [ecco.Tables(learn_tables(c, seed=0, npat=16), dev) for c in (Kc, Vc)]}
+        self.blocks = [torch.empty((self.n, 64), dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.launches_per_step = 2
+        self.enc_ms = []
+        self.quality = self._study()
+
+    def _study(self):
+        torch, ecco = self.torch, self.ecco
+        out, chosen = {}, {}
+        for npat in (64, 16):
+            for sel, sname in ((self._lib.SELECT_MINMAX, "minmax"), (self._lib.SELECT_MSE, "mse")):
+                err = ref = 0.0
+                ps = []
+                for i in range(2):
+                    t = self.tabs[npat][i]
+                    ecco.encode(self.x[i], t, out=self.blocks[i], select=sel, n_patterns=npat)
+                    torch.cuda.synchronize()
+                    a, b = _events(torch)
+                    a.record()
+                    ecco.encode(self.x[i], t, out=self.blocks[i], select=sel, n_patterns=npat)
+                    b.record()
+                    y = ecco.decode(self.blocks[i], t).float().view_as(self.x[i])
+                    xf = self.x[i].float()
+                    err += float(((y - xf) ** 2).sum())
+                    ref += float((xf ** 2).sum())
+                    ps.append((self.blocks[i][:, 1] & 63).clone())
+                    torch.cuda.synchronize()
+                    ms = a.elapsed_time(b)
+                    out.setdefault(f"{sname}{npat}", {"encode_GBps": []})["encode_GBps"].append(
+                        round(self.n * 256 / (ms * 1e-3) / 1e9, 1))
+                out[f"{sname}{npat}"]["rel_mse"] = err / ref
+                chosen[(sname, npat)] = torch.cat(ps)
+        for npat in (64, 16):
+            diff = (chosen[("minmax", npat)] != chosen[("mse", npat)]).float().mean().item()
+            out[f"minmax{npat}"]["pattern_differs_from_mse"] = round(diff, 4)
+        return out
+
+    def bytes_encoded(self):
+        return 2 * self.n * 256
+
+    def cpu_frac(self):
+        return 1.0 / 512
+
+    def step(self, record=False):
+        if record:
+            a, b = _events(self.torch)
+            a.record()
+        for i in range(2):
+            self.ecco.encode(self.x[i], self.tabs[64][i], out=self.blocks[i], select=self._lib.SELECT_MSE)
+        if record:
+            b.record()
+            self.enc_ms.append((a, b))
+
+    def dominant(self):
+        self.torch.cuda.synchronize()
+        return "encode_kernel<.,SEL=1>", 2 * self.n * 320, [a.elapsed_time(b) for a, b in self.enc_ms]
+
+    def per_op(self):
+        return {"selection_study": self.quality}
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.hx = [t.cpu().pin_memory() for t in self.x]
+        self.hb = [torch.empty((self.n, 64), dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self.dx = [torch.empty_like(t) for t in self.x]
+        self.h2d = sum(t.numel() * 2 for t in self.hx)
+        self.d2h = sum(t.numel() for t in self.hb)
+
+    def e2e_step(self):
+        for i in range(2):
+            self.dx[i].copy_(self.hx[i], non_blocking=True)
+            self.ecco.encode(self.dx[i], self.tabs[64][i], out=self.blocks[i], select=self._lib.SELECT_MSE)
+            self.hb[i].copy_(self.blocks[i], non_blocking=True)
+
+    def cpu_sample(self, frac):
+        import workloads as W
+        k = max(64, int(self.n * frac))
+        xs = [W.bf16_bits(self.x[i].view(-1, 128)[:k]) for i in range(2)]
+        return {"enc": [(self.tabs[64][i].blob, xs[i]) for i in range(2)], "dec": [],
+                "select": 1, "bytes": 2 * k * 256,
+                "what": f"full-MSE encode of {2 * k} groups (1/{round(1 / frac)} of a step)"}
+
+
 WORKLOADS = {"kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload, "model": ModelWorkload,
-             "longctx": LongCtxWorkload, "attn": AttnWorkload}
+             "longctx": LongCtxWorkload, "attn": AttnWorkload, "select": SelectWorkload}
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -668,7 +774,7 @@ def time_oracle(sample, nthreads):
     import oracle
     t0 = time.perf_counter()
     for blob, xb in sample["enc"]:
-        oracle.encode(blob, xb, nthreads=nthreads)
+        oracle.encode(blob, xb, nthreads=nthreads, select=sample.get("select", 0))
     for blob, bl in sample["dec"]:
         oracle.decode(blob, bl, nthreads=nthreads)
     if "attn" in sample:

@@ -96,9 +96,12 @@ def read_stats(stats: torch.Tensor) -> dict:
 
 
 def encode(x: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
-           stats: torch.Tensor | None = None, desc: Desc | None = None) -> torch.Tensor:
+           stats: torch.Tensor | None = None, desc: Desc | None = None, select: int = _lib.SELECT_MINMAX,
+           n_patterns: int = 64) -> torch.Tensor:
     """bf16 groups of 128 -> uint8 blocks [n_groups, 64].  With `desc`, `x` and
-    `out` are the full source / destination buffers the descriptor indexes."""
+    `out` are the full source / destination buffers the descriptor indexes.
+    `select` / `n_patterns` choose the pattern-selection variant
+    (ecco_select_encode_ex); the defaults are the method's own."""
     _check_tensor(x, torch.bfloat16, "x", tables.device)
     if desc is None:
         if x.numel() % GROUP:
@@ -111,9 +114,15 @@ def encode(x: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
     _check_tensor(out, torch.uint8, "out", tables.device)
     _bounds(desc, x.numel() // GROUP, out.numel() // BLOCK_BYTES)
     sp = ctypes.c_void_p(stats.data_ptr()) if stats is not None else None
-    rc = _lib.load().ecco_select_encode(tables.handle, ctypes.c_void_p(x.data_ptr()), desc,
-                                        ctypes.c_void_p(out.data_ptr()), sp, _stream(x.device))
-    _lib.check(rc, "ecco_select_encode")
+    if select == _lib.SELECT_MINMAX and n_patterns == 64:
+        rc = _lib.load().ecco_select_encode(tables.handle, ctypes.c_void_p(x.data_ptr()), desc,
+                                            ctypes.c_void_p(out.data_ptr()), sp, _stream(x.device))
+        _lib.check(rc, "ecco_select_encode")
+    else:
+        rc = _lib.load().ecco_select_encode_ex(tables.handle, ctypes.c_void_p(x.data_ptr()), desc,
+                                               ctypes.c_void_p(out.data_ptr()), sp, int(select), int(n_patterns),
+                                               _stream(x.device))
+        _lib.check(rc, "ecco_select_encode_ex")
     return out
 
 

@@ -17,6 +17,8 @@ ECCO_ERR_DEVICE = -5
 ECCO_ERR_UNSUPPORTED = -6
 ECCO_ERR_WORKSPACE = -7
 ATTENTION_STATIC_WS_BYTES = 4 << 20
+SELECT_MINMAX = 0
+SELECT_MSE = 1
 TABLES_BYTES = 7952
 MAX_SEGMENTS = 256
 
@@ -24,7 +26,7 @@ EXPORTED = [
     "ecco_tables_create", "ecco_tables_destroy", "ecco_select_encode", "ecco_decode",
     "ecco_decode_gemv", "ecco_decode_multi", "ecco_encode_multi", "ecco_strerror",
     "ecco_abi_version", "ecco_device_timeouts", "ecco_decode_attention",
-    "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static",
+    "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static", "ecco_select_encode_ex",
 ]
 
 
@@ -63,6 +65,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_tables_destroy.argtypes = [P]
     L.ecco_select_encode.argtypes = [P, P, Desc, P, P, P]
     L.ecco_decode.argtypes = [P, P, Desc, P, P]
+    L.ecco_select_encode_ex.argtypes = [P, P, Desc, P, P, I, I, P]
     L.ecco_decode_gemv.argtypes = [P, P, I64, I64, P, I, P, P]
     L.ecco_decode_multi.argtypes = [ctypes.POINTER(Segment), I, P]
     L.ecco_encode_multi.argtypes = [ctypes.POINTER(Segment), I, P, P]

@@ -130,8 +130,13 @@ def _quantise(u_rows, T_rows):
 
 
 def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
-                 refine_iters: int = 4, codebook_iters: int = 6) -> bytes:
-    """Learns a table blob from a bf16 (or float) sample whose numel % 128 == 0."""
+                 refine_iters: int = 4, codebook_iters: int = 6, npat: int = NPAT) -> bytes:
+    """Learns a table blob from a bf16 (or float) sample whose numel % 128 == 0.
+    npat < 64 learns that many patterns (the compressor's 16-pattern variant,
+    free parameters: "reduced from 64"); rows npat..63 repeat row 0 and are
+    never chosen by an encoder that searches npat patterns."""
+    if not 1 <= npat <= NPAT:
+        raise ValueError("npat must be in 1..64")
     X = sample.detach().float().reshape(-1, G).cpu().numpy().astype(np.float32)
     X = np.where(np.isfinite(X), X, 0).astype(np.float32)
     absmax = float(np.abs(X).max()) if X.size else 0.0
@@ -154,7 +159,7 @@ def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
     srt = np.sort(rest, axis=1)
     edges = np.linspace(0, G - 1, NCENT + 1).round().astype(int)
     F = np.stack([srt[:, edges[j]:edges[j + 1]].mean(1) for j in range(NCENT)], axis=1)
-    C = _kmeans(F, NPAT, rng)
+    C = _kmeans(F, npat, rng)
     C = np.stack([_strictly_increasing(c) for c in C])
 
     umin, umax = rest.min(1), rest.max(1)
@@ -162,7 +167,7 @@ def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
         p = _assign_minmax(umin, umax, C)
         T = _thresholds(C)
         sym = _quantise(rest, T[p])
-        for q in range(NPAT):
+        for q in range(npat):
             sel = p == q
             if not sel.any():
                 continue
@@ -183,7 +188,7 @@ def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
     hist[:, 15] = 1
     lens = np.zeros((NPAT, NBOOK, NSYM), dtype=np.uint8)
     glob_len = package_merge(hist.sum(0) + 1)
-    for q in range(NPAT):
+    for q in range(npat):
         Hq = hist[p == q]
         if len(Hq) == 0:
             lens[q, :] = glob_len
@@ -202,6 +207,9 @@ def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
                 books[h] = package_merge(Hq[sel].sum(0) + 1 if sel.any() else base)
             a = np.argmin(Hq @ books.T.astype(np.int64), axis=1)
         lens[q] = books
+    if npat < NPAT:
+        C = np.concatenate([C, np.repeat(C[:1], NPAT - npat, axis=0)])
+        lens[npat:] = lens[0]
     from struct import pack
     Cb = np.ascontiguousarray(C.astype(np.float32))
     blob = pack("<IIfI", TABLES_MAGIC, 1, float(S_t), 0) + Cb.tobytes() + np.ascontiguousarray(lens).tobytes()

@@ -61,7 +61,8 @@ namespace ecco {
 // ------------------------------------------------------------ launchers
 
 cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
-                          uint8_t* blocks, ecco_stats* stats, cudaStream_t s);
+                          uint8_t* blocks, ecco_stats* stats, cudaStream_t s,
+                          int select = ECCO_SELECT_MINMAX, int npat = kNPat);
 cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
                           uint16_t* y, cudaStream_t s);
 cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,

@@ -124,6 +124,24 @@ int ecco_tables_destroy(ecco_tables* tables);
 int ecco_select_encode(const ecco_tables* tables, const uint16_t* x_bf16, ecco_desc desc,
                        uint8_t* blocks, ecco_stats* dev_stats, void* stream);
 
+/* Encoder variants for studying the pattern choice.  `select`:
+ *   ECCO_SELECT_MINMAX  the method's min/max squared error (as ecco_select_encode);
+ *   ECCO_SELECT_MSE     the full squared error of the normalised group: for each
+ *                       pattern p, e_p = pairwise (binary-tree, element order)
+ *                       fp32 sum of (u_i - C[p][sym_p(u_i)])^2, the scale
+ *                       element adding 0; first p with the least e_p.  The
+ *                       comparison the review page's referee report asks for
+ *                       (major comment 2); about 10x the encoder's work.
+ * `n_patterns` (1..64): only patterns 0..n_patterns-1 are searched (free
+ * parameters: the compressor's 16 patterns, "reduced from 64"); tables for it
+ * are learned with that many patterns.  Blocks decode with ecco_decode as
+ * usual.  Other arguments as ecco_select_encode. */
+#define ECCO_SELECT_MINMAX 0
+#define ECCO_SELECT_MSE 1
+int ecco_select_encode_ex(const ecco_tables* tables, const uint16_t* x_bf16, ecco_desc desc,
+                          uint8_t* blocks, ecco_stats* dev_stats, int select, int n_patterns,
+                          void* stream);
+
 /* Decoder (the review page's decompressor, Fig. 8 caption): every block of
  * `blocks` described by `desc` becomes 128 bf16 values in `y_bf16`.  Any
  * 64-byte pattern decodes deterministically (malformed blocks included).
