@@ -120,6 +120,14 @@ def lib():
             L.or_decode_block.argtypes = [P, P, P]
             L.or_encode.restype = None
             L.or_encode.argtypes = [P, P, I64, P, P, ctypes.c_int, ctypes.c_int]
+            L.or_encode_group_gs.restype = None
+            L.or_encode_group_gs.argtypes = [P, P, P, P] + [ctypes.c_int] * 5
+            L.or_decode_block_gs.restype = ctypes.c_int
+            L.or_decode_block_gs.argtypes = [P, P, P, ctypes.c_int]
+            L.or_encode_gs.restype = None
+            L.or_encode_gs.argtypes = [P, P, I64, P, P] + [ctypes.c_int] * 5
+            L.or_decode_gs.restype = None
+            L.or_decode_gs.argtypes = [P, P, I64, P, ctypes.c_int, ctypes.c_int]
             L.or_encode_sel.restype = None
             L.or_encode_sel.argtypes = [P, P, I64, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
             L.or_decode.restype = None
@@ -186,55 +194,58 @@ def canonical_codes(tables, p: int, h: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- codec
+G_ACT = 64          # R25: activation groups (2x format)
 SELECT_MINMAX = 0   # R8: min/max squared error (the method)
 SELECT_MSE = 1      # R23: full squared error, pairwise fp32 sum
 
 
 def encode_group(tables, x, force_p: int = -1, force_h: int = -1, select: int = SELECT_MINMAX,
-                 npat: int = NPAT):
+                 npat: int = NPAT, gs: int = G):
     """One group: returns (block bytes [64] uint8, GroupInfo).  `select` and
-    `npat` (patterns searched, R24) pick the selection variant."""
+    `npat` (patterns searched, R24) pick the selection variant; gs = 64 is
+    the activation format (R25)."""
     b = _blob(tables)
     xb = _bits(x).reshape(-1)
-    assert xb.size == G and 1 <= npat <= NPAT
+    assert gs in (G, G_ACT) and xb.size == gs and 1 <= npat <= NPAT
     blk = np.zeros(BLOCK_BYTES, dtype=np.uint8)
     info = GroupInfo()
-    lib().or_encode_group_sel(_ptr(b), _ptr(xb), _ptr(blk), ctypes.byref(info), select, npat, force_p, force_h)
+    lib().or_encode_group_gs(_ptr(b), _ptr(xb), _ptr(blk), ctypes.byref(info), gs, select, npat, force_p, force_h)
     return blk, info
 
 
-def decode_block(tables, blk) -> tuple[np.ndarray, int]:
+def decode_block(tables, blk, gs: int = G) -> tuple[np.ndarray, int]:
     b = _blob(tables)
     bb = np.ascontiguousarray(np.asarray(blk, dtype=np.uint8).reshape(-1))
-    assert bb.size == BLOCK_BYTES
-    y = np.zeros(G, dtype=np.uint16)
-    k = lib().or_decode_block(_ptr(b), _ptr(bb), _ptr(y))
+    assert bb.size == BLOCK_BYTES and gs in (G, G_ACT)
+    y = np.zeros(gs, dtype=np.uint16)
+    k = lib().or_decode_block_gs(_ptr(b), _ptr(bb), _ptr(y), gs)
     return y, int(k)
 
 
 def encode(tables, x, with_mse: bool = False, nthreads: int = 1, select: int = SELECT_MINMAX,
-           npat: int = NPAT):
+           npat: int = NPAT, gs: int = G):
     """x: [..., 128*k] bf16 bits, contiguous groups.  Returns (blocks [n,64], Stats).
     With with_mse, Stats.mse_minmax is the fp64 squared error of the chosen
     patterns (whatever `select`), mse_full that of the fp64-best of all 64."""
     b = _blob(tables)
     xb = _bits(x).reshape(-1)
-    assert xb.size % G == 0 and 1 <= npat <= NPAT
-    n = xb.size // G
+    assert gs in (G, G_ACT) and xb.size % gs == 0 and 1 <= npat <= NPAT
+    n = xb.size // gs
     blocks = np.zeros((n, BLOCK_BYTES), dtype=np.uint8)
     st = Stats()
-    lib().or_encode_sel(_ptr(b), _ptr(xb), n, _ptr(blocks), ctypes.byref(st), int(with_mse), nthreads,
-                        select, npat)
+    lib().or_encode_gs(_ptr(b), _ptr(xb), n, _ptr(blocks), ctypes.byref(st), int(with_mse), nthreads,
+                       select, npat, gs)
     return blocks, st
 
 
-def decode(tables, blocks, nthreads: int = 1) -> np.ndarray:
-    """blocks: [n, 64] uint8.  Returns bf16 bits [n, 128] uint16."""
+def decode(tables, blocks, nthreads: int = 1, gs: int = G) -> np.ndarray:
+    """blocks: [n, 64] uint8.  Returns bf16 bits [n, gs] uint16."""
     b = _blob(tables)
     bb = np.ascontiguousarray(np.asarray(blocks, dtype=np.uint8).reshape(-1, BLOCK_BYTES))
+    assert gs in (G, G_ACT)
     n = bb.shape[0]
-    y = np.zeros((n, G), dtype=np.uint16)
-    lib().or_decode(_ptr(b), _ptr(bb), n, _ptr(y), nthreads)
+    y = np.zeros((n, gs), dtype=np.uint16)
+    lib().or_decode_gs(_ptr(b), _ptr(bb), n, _ptr(y), nthreads, gs)
     return y
 
 

@@ -55,6 +55,12 @@
  *       order, of d_i * d_i with d_i = u_i - C[p][sym_p(u_i)]; slot m adds +0.
  *       Pairwise = a perfect binary tree (slots 0..63 + slots 64..127, each
  *       half the same way).  Every op one fp32 rounding; first p with the least e_p.
+ *   R25 activation blocks (free parameters: "Group size for activations = 64",
+ *       "2x activations"; Fig. 9 text: the low-ratio compressor reuses the
+ *       high-ratio compressor's components): a group of 64 values becomes one
+ *       512-bit block with the same header, symbols, codebook choice, clipping
+ *       and padding rules (records keep the 15-bit layout; at most 16); the
+ *       decoder takes a record's 7-bit index modulo 64.
  *   R24 the compressor's pattern count (free parameters: "Shared k-means
  *       patterns used in the compressor = 16, reduced from 64"): selection
  *       searches patterns 0..npat-1 only; the block format is unchanged.
@@ -286,10 +292,10 @@ static int quantise(const or_tables* t, int p, float u)
 }
 
 /* Full squared error of the normalised group under pattern p (fp64 sum). */
-static double pattern_mse(const or_tables* t, int p, const float* u, int m)
+static double pattern_mse(const or_tables* t, int p, const float* u, int m, int gs)
 {
     double acc = 0.0;
-    for (int i = 0; i < OR_G; ++i) {
+    for (int i = 0; i < gs; ++i) {
         if (i == m) continue;
         double d = (double)u[i] - (double)t->C[p][quantise(t, p, u[i])];
         acc += d * d;
@@ -307,22 +313,22 @@ static float pairwise_sum(const float* v, int n)
 }
 
 /* R23: full squared error of the normalised group under pattern p. */
-static float pattern_sq_error(const or_tables* t, int p, const float* u, int m)
+static float pattern_sq_error(const or_tables* t, int p, const float* u, int m, int gs)
 {
     float d2[OR_G];
-    for (int i = 0; i < OR_G; ++i) {
+    for (int i = 0; i < gs; ++i) {
         if (i == m) { d2[i] = 0.0f; continue; }
         float d = u[i] - t->C[p][quantise(t, p, u[i])];
         d2[i] = d * d;
     }
-    return pairwise_sum(d2, OR_G);
+    return pairwise_sum(d2, gs);
 }
 
 /* select: 0 = min/max fitness (R8), 1 = full squared error (R23); npat = number
  * of patterns the selection searches (R24, 1..64).  force_p / force_h < 0: the
  * method's own choice; >= 0: forced (tests only). */
-void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
-                         or_group_info* info, int select, int npat, int force_p, int force_h)
+void or_encode_group_gs(const or_tables* t, const uint16_t* x_in, uint8_t* blk, or_group_info* info,
+                        int gs, int select, int npat, int force_p, int force_h)
 {
     or_group_info gi;
     memset(&gi, 0, sizeof gi);
@@ -330,14 +336,14 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
 
     /* R21: non-finite elements become +0. */
     uint16_t x[OR_G];
-    for (int i = 0; i < OR_G; ++i) {
+    for (int i = 0; i < gs; ++i) {
         x[i] = x_in[i];
         if ((x[i] & 0x7f80u) == 0x7f80u) { x[i] = 0; gi.nonfinite += 1; }
     }
 
     /* R4: first index of the largest magnitude. */
     int m = 0;
-    for (int i = 1; i < OR_G; ++i)
+    for (int i = 1; i < gs; ++i)
         if ((x[i] & 0x7fffu) > (x[m] & 0x7fffu)) m = i;
     gi.m = m;
 
@@ -346,11 +352,11 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
     uint8_t code = or_e4m3_from_f32(r);
     double fp8v = or_e4m3_value(code);
     gi.code = code;
-    gi.k_clip = OR_G;
+    gi.k_clip = gs;
     if (fp8v == 0.0) { /* R7 */
         gi.zero = 1;
         gi.code = 0;
-        for (int i = 0; i < OR_G; ++i) gi.sym[i] = 0;
+        for (int i = 0; i < gs; ++i) gi.sym[i] = 0;
         if (info) *info = gi;
         return;
     }
@@ -361,12 +367,12 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
 
     /* R6 */
     float u[OR_G];
-    for (int i = 0; i < OR_G; ++i) u[i] = (i == m) ? 0.0f : or_bf16_to_f32(x[i]) * inv;
+    for (int i = 0; i < gs; ++i) u[i] = (i == m) ? 0.0f : or_bf16_to_f32(x[i]) * inv;
     memcpy(gi.u, u, sizeof u);
 
     /* R8: min/max pattern fitness. */
     float umin = INFINITY, umax = -INFINITY;
-    for (int i = 0; i < OR_G; ++i) {
+    for (int i = 0; i < gs; ++i) {
         if (i == m) continue;
         if (u[i] < umin) umin = u[i];
         if (u[i] > umax) umax = u[i];
@@ -383,7 +389,7 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
             float sq1 = d1 * d1;
             e = sq0 + sq1;
         } else {
-            e = pattern_sq_error(t, q, u, m);
+            e = pattern_sq_error(t, q, u, m, gs);
         }
         gi.e[q] = e;
         if (e < gi.e[p]) p = q;
@@ -392,13 +398,13 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
     gi.p = (uint8_t)p;
 
     /* R5, R9 */
-    for (int i = 0; i < OR_G; ++i) gi.sym[i] = (uint8_t)((i == m) ? 15 : quantise(t, p, u[i]));
+    for (int i = 0; i < gs; ++i) gi.sym[i] = (uint8_t)((i == m) ? 15 : quantise(t, p, u[i]));
 
     /* R13: shortest codebook over the whole group. */
     int h = 0;
     for (int b = 0; b < OR_NBOOK; ++b) {
         int L = 0;
-        for (int i = 0; i < OR_G; ++i) L += t->len[p][b][gi.sym[i]];
+        for (int i = 0; i < gs; ++i) L += t->len[p][b][gi.sym[i]];
         gi.Lh[b] = L;
         if (L < gi.Lh[h]) h = b;
     }
@@ -415,15 +421,15 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
     canonical_codes(t->len[p][h], cw);
     int pos = OR_HDR_BITS;
     int L = 0;
-    for (int i = 0; i < OR_G; ++i) {
+    for (int i = 0; i < gs; ++i) {
         int l = t->len[p][h][gi.sym[i]];
-        if (pos + l > OR_BLOCK_BITS && gi.k_clip == OR_G) gi.k_clip = i;
+        if (pos + l > OR_BLOCK_BITS && gi.k_clip == gs) gi.k_clip = i;
         if (pos < OR_BLOCK_BITS) put_codeword(blk, pos, cw[gi.sym[i]], l);
         pos += l;
         L += l;
     }
     gi.L = L;
-    gi.clipped = (gi.k_clip < OR_G);
+    gi.clipped = (gi.k_clip < gs);
 
     /* R15, R16: outlier records in the spare bits. */
     if (!gi.clipped) {
@@ -434,7 +440,7 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
         taken[m] = 1;
         for (int k = 0; k < n; ++k) {
             int best = -1;
-            for (int i = 0; i < OR_G; ++i) {
+            for (int i = 0; i < gs; ++i) {
                 if (taken[i]) continue;
                 if (best < 0 || (x[i] & 0x7fffu) > (x[best] & 0x7fffu)) best = i;
             }
@@ -453,6 +459,12 @@ void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
         gi.n_rec = n;
     }
     if (info) *info = gi;
+}
+
+void or_encode_group_sel(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
+                         or_group_info* info, int select, int npat, int force_p, int force_h)
+{
+    or_encode_group_gs(t, x_in, blk, info, OR_G, select, npat, force_p, force_h);
 }
 
 void or_encode_group_ex(const or_tables* t, const uint16_t* x_in, uint8_t* blk,
@@ -485,9 +497,9 @@ static int read_codeword(const uint8_t* blk, int* pos, const uint8_t len[OR_NSYM
 }
 
 /* Returns the number of elements decoded from codewords (128 unless clipped). */
-int or_decode_block(const or_tables* t, const uint8_t* blk, uint16_t* y)
+int or_decode_block_gs(const or_tables* t, const uint8_t* blk, uint16_t* y, int gs)
 {
-    for (int i = 0; i < OR_G; ++i) y[i] = 0;
+    for (int i = 0; i < gs; ++i) y[i] = 0;
     uint8_t code = (uint8_t)get_field(blk, 0, 8);
     int p = (int)get_field(blk, 8, 6);
     int h = (int)get_field(blk, 14, 2);
@@ -499,25 +511,30 @@ int or_decode_block(const or_tables* t, const uint8_t* blk, uint16_t* y)
     canonical_codes(t->len[p][h], cw);
     int pos = OR_HDR_BITS;
     int k = 0;
-    for (; k < OR_G; ++k) {
+    for (; k < gs; ++k) {
         int sym = read_codeword(blk, &pos, t->len[p][h], cw);
         if (sym < 0) break;
         float c = (sym == 15) ? 1.0f : t->C[p][sym];
         y[k] = or_f32_to_bf16(s * c);
     }
-    if (k == OR_G) {
+    if (k == gs) {
         int L = pos - OR_HDR_BITS;
         int n = (OR_PAYLOAD_BITS - L) / OR_REC_BITS;
         if (n > OR_MAX_REC) n = OR_MAX_REC;
         for (int r = 0; r < n; ++r) {
             int at = pos + r * OR_REC_BITS;
-            int i = (int)get_field(blk, at, 7);
+            int i = (int)get_field(blk, at, 7) % gs; /* R18, R25 */
             int q = (int)(int8_t)(uint8_t)get_field(blk, at + 7, 8);
             float o = (float)q / 127.0f;
             y[i] = or_f32_to_bf16(s * o);
         }
     }
     return k;
+}
+
+int or_decode_block(const or_tables* t, const uint8_t* blk, uint16_t* y)
+{
+    return or_decode_block_gs(t, blk, y, OR_G);
 }
 
 /* ------------------------------------------------------------------ */
@@ -531,7 +548,7 @@ typedef struct {
     uint16_t* y;
     int64_t lo, hi;
     int with_mse;
-    int select, npat;
+    int select, npat, gs;
     or_stats st;
 } or_job;
 
@@ -540,8 +557,8 @@ static void* encode_worker(void* arg)
     or_job* j = (or_job*)arg;
     or_group_info gi;
     for (int64_t g = j->lo; g < j->hi; ++g) {
-        or_encode_group_sel(j->t, j->x + g * OR_G, j->blocks + g * OR_BLOCK_BYTES, &gi, j->select, j->npat,
-                            -1, -1);
+        or_encode_group_gs(j->t, j->x + g * j->gs, j->blocks + g * OR_BLOCK_BYTES, &gi, j->gs, j->select,
+                           j->npat, -1, -1);
         j->st.n_groups += 1;
         j->st.n_nonfinite += (uint64_t)gi.nonfinite;
         if (gi.zero) { j->st.n_zero += 1; continue; }
@@ -557,11 +574,11 @@ static void* encode_worker(void* arg)
             int pbest = 0;
             double ebest = INFINITY;
             for (int p = 0; p < OR_NPAT; ++p) {
-                double e = pattern_mse(j->t, p, gi.u, gi.m);
+                double e = pattern_mse(j->t, p, gi.u, gi.m, j->gs);
                 if (e < ebest) { ebest = e; pbest = p; }
             }
             j->st.mse_full += ebest;
-            j->st.mse_minmax += pattern_mse(j->t, gi.p, gi.u, gi.m);
+            j->st.mse_minmax += pattern_mse(j->t, gi.p, gi.u, gi.m, j->gs);
             if (pbest != gi.p) j->st.n_mse_differs += 1;
         }
     }
@@ -572,7 +589,7 @@ static void* decode_worker(void* arg)
 {
     or_job* j = (or_job*)arg;
     for (int64_t g = j->lo; g < j->hi; ++g)
-        or_decode_block(j->t, j->blocks + g * OR_BLOCK_BYTES, j->y + g * OR_G);
+        or_decode_block_gs(j->t, j->blocks + g * OR_BLOCK_BYTES, j->y + g * j->gs, j->gs);
     return NULL;
 }
 
@@ -611,11 +628,12 @@ static void run_jobs(void* (*fn)(void*), or_job* base, int64_t n, int nthreads, 
 }
 
 /* x: n_groups * 128 bf16, contiguous; blocks: n_groups * 64 bytes. */
-void or_encode_sel(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
-                   or_stats* stats, int with_mse, int nthreads, int select, int npat)
+void or_encode_gs(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
+                  or_stats* stats, int with_mse, int nthreads, int select, int npat, int gs)
 {
     or_job base;
     memset(&base, 0, sizeof base);
+    base.gs = gs;
     base.t = t;
     base.x = x;
     base.blocks = blocks;
@@ -625,21 +643,34 @@ void or_encode_sel(const or_tables* t, const uint16_t* x, int64_t n_groups, uint
     run_jobs(encode_worker, &base, n_groups, nthreads, stats);
 }
 
+void or_encode_sel(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
+                   or_stats* stats, int with_mse, int nthreads, int select, int npat)
+{
+    or_encode_gs(t, x, n_groups, blocks, stats, with_mse, nthreads, select, npat, OR_G);
+}
+
 void or_encode(const or_tables* t, const uint16_t* x, int64_t n_groups, uint8_t* blocks,
                or_stats* stats, int with_mse, int nthreads)
 {
     or_encode_sel(t, x, n_groups, blocks, stats, with_mse, nthreads, 0, OR_NPAT);
 }
 
-void or_decode(const or_tables* t, const uint8_t* blocks, int64_t n_blocks, uint16_t* y,
-               int nthreads)
+void or_decode_gs(const or_tables* t, const uint8_t* blocks, int64_t n_blocks, uint16_t* y,
+                  int nthreads, int gs)
 {
     or_job base;
     memset(&base, 0, sizeof base);
+    base.gs = gs;
     base.t = t;
     base.blocks = (uint8_t*)blocks;
     base.y = y;
     run_jobs(decode_worker, &base, n_blocks, nthreads, NULL);
+}
+
+void or_decode(const or_tables* t, const uint8_t* blocks, int64_t n_blocks, uint16_t* y,
+               int nthreads)
+{
+    or_decode_gs(t, blocks, n_blocks, y, nthreads, OR_G);
 }
 
 /* y[b][r] = sum_k W~[r][k] * x[b][k] in fp64, W~ the decoded blocks of a row-major

@@ -68,10 +68,10 @@ RAMP = [0x0000, 0xBF60, 0xBF40, 0xBF20, 0xBF00, 0xBEC0, 0xBE80, 0xBE00,
 # RAMP[j + 1] is (j - 7) / 8 in bf16, j = 0..14 (RAMP[0] unused)
 
 
-def expand(spec) -> np.ndarray:
-    out = np.full(128, spec.get("rest", 0), dtype=np.uint16)
+def expand(spec, n: int = 128) -> np.ndarray:
+    out = np.full(n, spec.get("rest", 0), dtype=np.uint16)
     if spec.get("i_mod_15_ramp"):
-        for i in range(1, 128):
+        for i in range(1, n):
             out[i] = RAMP[(i % 15) + 1]
     if "i_mod_15_ramp_upto" in spec:
         for i in range(1, spec["i_mod_15_ramp_upto"] + 1):
@@ -117,8 +117,9 @@ def canonical_dict(lens):
     return table
 
 
-def ref_decode(blob: bytes, blk: np.ndarray) -> np.ndarray:
-    """Independent decoder of one block (format readings R1, R2, R7, R14, R15, R17, R18)."""
+def ref_decode(blob: bytes, blk: np.ndarray, gs: int = 128) -> np.ndarray:
+    """Independent decoder of one block (format readings R1, R2, R7, R14, R15,
+    R17, R18; gs = 64: the activation format, R25)."""
     _, _, S_t, C, lens = W.unpack_tables(blob)
     bits = np.unpackbits(np.asarray(blk, dtype=np.uint8), bitorder="little")
 
@@ -126,7 +127,7 @@ def ref_decode(blob: bytes, blk: np.ndarray) -> np.ndarray:
         return int(sum(int(bits[at + i]) << i for i in range(w)))
 
     code, p, h = field(0, 8), field(8, 6), field(14, 2)
-    y = np.zeros(128, dtype=np.uint16)
+    y = np.zeros(gs, dtype=np.uint16)
     v = e4m3_torch(code)
     if v == 0 or np.isnan(v):
         return y
@@ -134,7 +135,7 @@ def ref_decode(blob: bytes, blk: np.ndarray) -> np.ndarray:
     table = canonical_dict(lens[p, h])
     pos, k, cur = 16, 0, ""
     vals = []
-    while k < 128 and pos < 512:
+    while k < gs and pos < 512:
         cur += str(int(bits[pos]))
         pos += 1
         if cur in table:
@@ -144,12 +145,12 @@ def ref_decode(blob: bytes, blk: np.ndarray) -> np.ndarray:
             k += 1
             cur = ""
     y[: len(vals)] = f32_to_bf16_torch(np.array(vals, dtype=np.float32)) if vals else y[:0]
-    if k == 128:
+    if k == gs:
         L = pos - 16
         n = min(16, (496 - L) // 15)
         for r in range(n):
             at = pos + 15 * r
-            i = field(at, 7)
+            i = field(at, 7) % gs
             q = field(at + 7, 8)
             q = q - 256 if q >= 128 else q
             o = np.float32(q) / np.float32(127.0)
@@ -162,9 +163,10 @@ def ref_decode(blob: bytes, blk: np.ndarray) -> np.ndarray:
 def test_golden_encode(name):
     blob, spec = golden_tables()
     case = next(c for c in spec["cases"] if c["name"] == name)
-    x = expand(case["x"])
+    gs = case.get("group", 128)
+    x = expand(case["x"], gs)
     want = assemble_stream(case["stream"])
-    got, info = oracle.encode_group(blob, x)
+    got, info = oracle.encode_group(blob, x, gs=gs)
     assert got.tobytes().hex() == want.tobytes().hex()
     assert info.nonfinite == case.get("nonfinite", 0)
 
@@ -174,10 +176,11 @@ def test_golden_decode(name):
     blob, spec = golden_tables()
     case = next(c for c in spec["cases"] if c["name"] == name)
     blk = assemble_stream(case["stream"])
-    want = expand(case["decoded"])
-    got, _ = oracle.decode_block(blob, blk)
+    gs = case.get("group", 128)
+    want = expand(case["decoded"], gs)
+    got, _ = oracle.decode_block(blob, blk, gs=gs)
     np.testing.assert_array_equal(got, want)
-    np.testing.assert_array_equal(ref_decode(blob, blk), want)
+    np.testing.assert_array_equal(ref_decode(blob, blk, gs), want)
 
 
 def test_golden_canonical_codes():
@@ -304,24 +307,24 @@ def test_canonical_codes_prefix_free_and_ordered(seed):
 
 
 # ---------------------------------------------------------------- encoder decisions
-def random_group(rng, kind: int) -> np.ndarray:
+def random_group(rng, kind: int, n: int = 128) -> np.ndarray:
     if kind == 0:
-        v = rng.standard_normal(128) * 0.02
+        v = rng.standard_normal(n) * 0.02
     elif kind == 1:
-        v = rng.standard_t(5, 128) * 0.02
+        v = rng.standard_t(5, n) * 0.02
     elif kind == 2:
-        v = rng.standard_normal(128) * np.exp(rng.standard_normal(128) * 0.5)
-        v[rng.choice(128, 4, replace=False)] *= 15
+        v = rng.standard_normal(n) * np.exp(rng.standard_normal(n) * 0.5)
+        v[rng.choice(n, 4, replace=False)] *= 15
     else:
-        v = rng.standard_normal(128) * 0.02
-        v[rng.integers(128)] = rng.choice([-0.4, 0.4])
+        v = rng.standard_normal(n) * 0.02
+        v[rng.integers(n)] = rng.choice([-0.4, 0.4])
     return f32_to_bf16_torch(v.astype(np.float32))
 
 
-def check_group(blob, x):
+def check_group(blob, x, gs: int = 128):
     """Every decision of the oracle for one group, recomputed independently."""
     _, _, S_t, C, lens = W.unpack_tables(blob)
-    blk, gi = oracle.encode_group(blob, x)
+    blk, gi = oracle.encode_group(blob, x, gs=gs)
     xb = np.asarray(x, dtype=np.uint16).copy()
     xb[(xb & 0x7F80) == 0x7F80] = 0
     mag = xb & 0x7FFF
@@ -338,7 +341,7 @@ def check_group(blob, x):
     inv = np.float32(1.0) / s
     assert gi.s == s and gi.inv == inv
     u = bf16_to_f32_np(xb) * inv
-    others = np.array([i for i in range(128) if i != m])
+    others = np.array([i for i in range(gs) if i != m])
     assert np.array_equal(np.array(gi.u)[others], u[others])
     umin, umax = u[others].min(), u[others].max()
     assert gi.umin == umin and gi.umax == umax
@@ -355,7 +358,7 @@ def check_group(blob, x):
             assert gi.sym[i] == best, (i, gi.sym[i], best)
     assert gi.sym[m] == 15
     # codebook: shortest total length, first of ties
-    syms = np.array(gi.sym[:], dtype=np.int64)
+    syms = np.array(gi.sym[:gs], dtype=np.int64)
     Lh = lens[gi.p][:, syms].sum(axis=1)
     assert gi.h == int(np.argmin(Lh)) and gi.L == Lh[gi.h]
     # clipping / padding rules
@@ -370,7 +373,7 @@ def check_group(blob, x):
         assert gi.L + 15 * n <= 496
         if n < 16:
             assert 496 - gi.L - 15 * n < 15
-        rank = sorted([i for i in range(128) if i != m], key=lambda i: (-int(mag[i]), i))[:n]
+        rank = sorted([i for i in range(gs) if i != m], key=lambda i: (-int(mag[i]), i))[:n]
         assert list(gi.rec_pos[:n]) == rank
         for k, i in enumerate(rank):
             q = int(np.clip(np.rint(np.float32(u[i]) * np.float32(127.0)), -127, 127))
@@ -555,3 +558,49 @@ def test_min_max_exclude_the_scale_element():
     _, gi = oracle.encode_group(W.pack_tables(S_t, C2, lens), x)
     assert gi.umin == np.float32(0.25) and gi.umax == u3
     assert gi.p == 30
+
+
+# ---------------------------------------------------------------- activation format (R25)
+@pytest.mark.parametrize("seed", [0, 1])
+def test_activation_groups_encoder_decisions(seed):
+    rng = np.random.default_rng(300 + seed)
+    blob = W.random_tables(60 + seed, S_t=float(rng.uniform(1e-4, 3e-3)))
+    for it in range(200):
+        check_group(blob, random_group(rng, it % 4, 64), gs=64)
+
+
+def test_activation_round_trip_and_garbage_blocks():
+    rng = np.random.default_rng(310)
+    blob = W.random_tables(70, S_t=0.02 * 4 / 448)
+    _, _, S_t, C, lens = W.unpack_tables(blob)
+    for it in range(120):
+        x = random_group(rng, it % 4, 64)
+        blk, gi = oracle.encode_group(blob, x, gs=64)
+        y, k = oracle.decode_block(blob, blk, gs=64)
+        np.testing.assert_array_equal(y, ref_decode(blob, blk, 64))
+        if gi.zero:
+            continue
+        cp = np.concatenate([C[gi.p], [np.float32(1.0)]]).astype(np.float32)
+        want = f32_to_bf16_torch(np.float32(gi.s) * cp[np.array(gi.sym[:64])])
+        want[gi.k_clip:] = 0
+        for r in range(gi.n_rec):
+            o = np.float32(gi.rec_q[r]) / np.float32(127.0)
+            want[gi.rec_pos[r]] = f32_to_bf16_torch([np.float32(gi.s) * o])[0]
+        np.testing.assert_array_equal(y, want)
+    for _ in range(300):  # record indexes >= 64 wrap (R25)
+        blk = rng.integers(0, 256, 64, dtype=np.uint8)
+        np.testing.assert_array_equal(oracle.decode_block(blob, blk, gs=64)[0], ref_decode(blob, blk, 64))
+
+
+def test_activation_batch_entry_points():
+    rng = np.random.default_rng(320)
+    blob = W.random_tables(71, S_t=0.02 * 4 / 448)
+    xs = np.stack([random_group(rng, i % 4, 64) for i in range(96)])
+    blocks, st = oracle.encode(blob, xs, nthreads=3, gs=64)
+    for i in range(96):
+        np.testing.assert_array_equal(blocks[i], oracle.encode_group(blob, xs[i], gs=64)[0])
+    y = oracle.decode(blob, blocks, nthreads=2, gs=64)
+    assert y.shape == (96, 64)
+    for i in range(96):
+        np.testing.assert_array_equal(y[i], oracle.decode_block(blob, blocks[i], gs=64)[0])
+    assert st.n_groups == 96
