@@ -13,7 +13,8 @@ encode and decode of the whole set), `longctx` (32 layers x K,V x
 `attn` (one-token append + fused decode+attention over the compressed cache of
 the `kv` layer, 32 query heads), `select` (encode of the `kv` layer with
 full-MSE pattern selection, plus a quality study of min/max vs full-MSE
-selection with 64 and 16 patterns).
+selection with 64 and 16 patterns), `act` (the 2x activation format: [8192,
+4096] hidden states in 64-value groups, encode + decode).
 
 Prints ONE JSON line (rank 0).  `value` is whole-job bf16 GB/s: bf16 bytes the
 step decodes plus bf16 bytes it encodes, over all ranks, per second of device
@@ -44,7 +45,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ecco", choices=["ecco", "reference"])
-    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select"])
+    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select", "act"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
@@ -765,7 +766,77 @@ class SelectWorkload(Workload):
                 "what": f"full-MSE encode of {2 * k} groups (1/{round(1 / frac)} of a step)"}
 
 
-WORKLOADS = {"kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload, "model": ModelWorkload,
+class ActWorkload(Workload):
+    """Activation format: [8192, 4096] bf16 hidden states (Llama-3-8B width) in
+    64-value groups; a step encodes and decodes all 524,288 groups."""
+    name = "act"
+    T, D, GA = 8192, 4096, 64
+
+    def __init__(self, dev, seed_offset=0):
+        import torch
+        import workloads as W
+        import entropy_coded_kv_b200 as ecco
+        from entropy_coded_kv_b200.calib import learn_tables
+        self.torch, self.ecco, self.dev = torch, ecco, dev
+        self.desc = ("activations [8192, 4096] bf16 (channel-outlier hidden states) in the 2x format: "
+                     "64-value groups, 524,288 blocks; encode + decode")
+        self.x = W.hidden_states(self.T, self.D, seed=6 + seed_offset, device=dev)
+        self.tables = ecco.Tables(learn_tables(W.hidden_states(2048, self.D, seed=61 + seed_offset),
+                                               seed=0, group=self.GA), dev)
+        self.n = self.x.numel() // self.GA
+        self.blocks = ecco.encode_act(self.x, self.tables)
+        self.out = torch.empty((self.n, self.GA), dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = 2
+        self.dec_ms = []
+
+    def bytes_decoded(self):
+        return self.n * self.GA * 2
+
+    def bytes_encoded(self):
+        return self.n * self.GA * 2
+
+    def cpu_frac(self):
+        return 1.0 / 64
+
+    def step(self, record=False):
+        self.ecco.encode_act(self.x, self.tables, out=self.blocks)
+        if record:
+            a, b = _events(self.torch)
+            a.record()
+        self.ecco.decode_act(self.blocks, self.tables, out=self.out)
+        if record:
+            b.record()
+            self.dec_ms.append((a, b))
+
+    def dominant(self):
+        self.torch.cuda.synchronize()
+        return "decode_kernel<G=64>", self.n * (64 + 128), [a.elapsed_time(b) for a, b in self.dec_ms]
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.hx = self.x.cpu().pin_memory()
+        self.hy = torch.empty((self.n, self.GA), dtype=torch.bfloat16).pin_memory()
+        self.dx = torch.empty_like(self.x)
+        self.h2d, self.d2h = self.hx.numel() * 2, self.hy.numel() * 2
+        self.api = "entropy_coded_kv_b200.encode_act/decode_act (C ABI) with pinned host buffers"
+
+    def e2e_step(self):
+        self.dx.copy_(self.hx, non_blocking=True)
+        self.ecco.encode_act(self.dx, self.tables, out=self.blocks)
+        self.ecco.decode_act(self.blocks, self.tables, out=self.out)
+        self.hy.copy_(self.out, non_blocking=True)
+
+    def cpu_sample(self, frac):
+        import workloads as W
+        k = max(64, int(self.n * frac))
+        xb = W.bf16_bits(self.x.view(-1, self.GA)[:k])
+        bl = self.blocks[:k].cpu().numpy()
+        return {"enc": [(self.tables.blob, xb)], "dec": [(self.tables.blob, bl)], "gs": self.GA,
+                "bytes": 2 * k * self.GA * 2,
+                "what": f"encode + decode of {k} activation groups (1/{round(1 / frac)} of a step)"}
+
+
+WORKLOADS = {"act": ActWorkload, "kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload, "model": ModelWorkload,
              "longctx": LongCtxWorkload, "attn": AttnWorkload, "select": SelectWorkload}
 
 
@@ -773,10 +844,11 @@ WORKLOADS = {"kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload, "model": Mo
 def time_oracle(sample, nthreads):
     import oracle
     t0 = time.perf_counter()
+    gs = sample.get("gs", 128)
     for blob, xb in sample["enc"]:
-        oracle.encode(blob, xb, nthreads=nthreads, select=sample.get("select", 0))
+        oracle.encode(blob, xb, nthreads=nthreads, select=sample.get("select", 0), gs=gs)
     for blob, bl in sample["dec"]:
-        oracle.decode(blob, bl, nthreads=nthreads)
+        oracle.decode(blob, bl, nthreads=nthreads, gs=gs)
     if "attn" in sample:
         (kt, vt), (kb, vb), qb, S, scale = sample["attn"]
         n = kb.shape[0]

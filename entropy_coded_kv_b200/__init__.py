@@ -20,10 +20,12 @@ from . import _lib
 from ._lib import EccoError, Desc, Segment, STATS_FIELDS
 
 GROUP = 128
+GROUP_ACT = 64  # activation format: 64 values per 64-byte block
 BLOCK_BYTES = 64
 
 __all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
            "decode_attention", "attention_workspace_bytes", "decode_attention_static",
+           "encode_act", "decode_act", "GROUP_ACT",
            "new_stats", "read_stats", "flat_desc", "kv_append_desc", "EccoError", "Desc"]
 
 
@@ -223,6 +225,44 @@ def decode_attention_static(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_ta
         ctypes.c_void_p(v_blocks.data_ptr()), s_cap, B, H, G, int(seq_len), ctypes.c_void_p(q.data_ptr()),
         float(scale), ctypes.c_void_p(out.data_ptr()), _stream(q.device))
     _lib.check(rc, "ecco_decode_attention_static")
+    return out
+
+
+def encode_act(x: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
+               stats: torch.Tensor | None = None, desc: Desc | None = None) -> torch.Tensor:
+    """Activation format: bf16 groups of 64 -> uint8 blocks [n_groups, 64]."""
+    _check_tensor(x, torch.bfloat16, "x", tables.device)
+    if desc is None:
+        if x.numel() % GROUP_ACT:
+            raise ValueError("x.numel() must be a multiple of 64")
+        desc = flat_desc(x.numel() // GROUP_ACT)
+    if out is None:
+        if desc.rows * desc.groups_per_row != x.numel() // GROUP_ACT or desc.dst_offset:
+            raise ValueError("pass `out` when the descriptor does not map x one-to-one")
+        out = torch.empty((x.numel() // GROUP_ACT, BLOCK_BYTES), dtype=torch.uint8, device=x.device)
+    _check_tensor(out, torch.uint8, "out", tables.device)
+    _bounds(desc, x.numel() // GROUP_ACT, out.numel() // BLOCK_BYTES)
+    sp = ctypes.c_void_p(stats.data_ptr()) if stats is not None else None
+    rc = _lib.load().ecco_select_encode_act(tables.handle, ctypes.c_void_p(x.data_ptr()), desc,
+                                            ctypes.c_void_p(out.data_ptr()), sp, _stream(x.device))
+    _lib.check(rc, "ecco_select_encode_act")
+    return out
+
+
+def decode_act(blocks: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
+               desc: Desc | None = None) -> torch.Tensor:
+    """Activation format: uint8 blocks [n, 64] -> bf16 [n, 64]."""
+    _check_tensor(blocks, torch.uint8, "blocks", tables.device)
+    n_blocks = blocks.numel() // BLOCK_BYTES
+    if desc is None:
+        desc = flat_desc(n_blocks)
+    if out is None:
+        out = torch.empty((desc.rows * desc.groups_per_row, GROUP_ACT), dtype=torch.bfloat16, device=blocks.device)
+    _check_tensor(out, torch.bfloat16, "out", tables.device)
+    _bounds(desc, n_blocks, out.numel() // GROUP_ACT)
+    rc = _lib.load().ecco_decode_act(tables.handle, ctypes.c_void_p(blocks.data_ptr()), desc,
+                                     ctypes.c_void_p(out.data_ptr()), _stream(blocks.device))
+    _lib.check(rc, "ecco_decode_act")
     return out
 
 

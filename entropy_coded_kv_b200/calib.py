@@ -68,7 +68,7 @@ def _e4m3_round(r: np.ndarray) -> np.ndarray:
 
 
 def normalise_groups(X: np.ndarray, S_t: np.float32):
-    """Scaled groups: returns (u [n, 128] fp32, m [n], keep mask)."""
+    """Scaled groups: returns (u [n, group] fp32, m [n], keep mask)."""
     mag = np.abs(X)
     m = np.argmax(mag, axis=1)
     xm = X[np.arange(len(X)), m]
@@ -130,14 +130,17 @@ def _quantise(u_rows, T_rows):
 
 
 def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
-                 refine_iters: int = 4, codebook_iters: int = 6, npat: int = NPAT) -> bytes:
+                 refine_iters: int = 4, codebook_iters: int = 6, npat: int = NPAT, group: int = G) -> bytes:
     """Learns a table blob from a bf16 (or float) sample whose numel % 128 == 0.
     npat < 64 learns that many patterns (the compressor's 16-pattern variant,
     free parameters: "reduced from 64"); rows npat..63 repeat row 0 and are
-    never chosen by an encoder that searches npat patterns."""
+    never chosen by an encoder that searches npat patterns.  group = 64 learns
+    tables for the activation format (64-value groups, same blob layout)."""
+    if group not in (G, 64):
+        raise ValueError("group must be 128 or 64")
     if not 1 <= npat <= NPAT:
         raise ValueError("npat must be in 1..64")
-    X = sample.detach().float().reshape(-1, G).cpu().numpy().astype(np.float32)
+    X = sample.detach().float().reshape(-1, group).cpu().numpy().astype(np.float32)
     X = np.where(np.isfinite(X), X, 0).astype(np.float32)
     absmax = float(np.abs(X).max()) if X.size else 0.0
     S_t = np.float32(absmax / 448.0) if absmax > 0 else np.float32(1.0)
@@ -149,15 +152,16 @@ def learn_tables(sample: torch.Tensor, seed: int = 0, max_groups: int = 16384,
     u, m = u[keep], m[keep]
     n = len(u)
     if n < NPAT:
-        u = np.concatenate([u, np.zeros((NPAT - n + 1, G), np.float32)]) if n else np.zeros((NPAT + 1, G), np.float32)
+        u = (np.concatenate([u, np.zeros((NPAT - n + 1, group), np.float32)]) if n
+             else np.zeros((NPAT + 1, group), np.float32))
         m = np.concatenate([m, np.zeros(len(u) - n, np.int64)]) if n else np.zeros(len(u), np.int64)
         n = len(u)
     mask = np.ones_like(u, dtype=bool)
     mask[np.arange(n), m] = False
-    rest = u[mask].reshape(n, G - 1)
+    rest = u[mask].reshape(n, group - 1)
 
     srt = np.sort(rest, axis=1)
-    edges = np.linspace(0, G - 1, NCENT + 1).round().astype(int)
+    edges = np.linspace(0, group - 1, NCENT + 1).round().astype(int)
     F = np.stack([srt[:, edges[j]:edges[j + 1]].mean(1) for j in range(NCENT)], axis=1)
     C = _kmeans(F, npat, rng)
     C = np.stack([_strictly_increasing(c) for c in C])

@@ -86,6 +86,31 @@ extern "C" int ecco_select_encode_ex(const ecco_tables* t, const uint16_t* x, ec
     return status(launch_encode(t, x, d, blocks, stats, (cudaStream_t)stream, select, n_patterns));
 }
 
+extern "C" int ecco_select_encode_act(const ecco_tables* t, const uint16_t* x, ecco_desc d, uint8_t* blocks,
+                                      ecco_stats* stats, void* stream)
+{
+    int rc = check_tables(t);
+    if (rc) return rc;
+    if ((rc = check_desc(d))) return rc;
+    if (d.rows == 0 || d.groups_per_row == 0) return ECCO_OK;
+    if (!x || !blocks) return ECCO_ERR_ARG;
+    if (!aligned16(x) || !aligned16(blocks) || (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return ECCO_ERR_ALIGN;
+    return status(launch_encode_act(t, x, d, blocks, stats, (cudaStream_t)stream));
+}
+
+extern "C" int ecco_decode_act(const ecco_tables* t, const uint8_t* blocks, ecco_desc d, uint16_t* y,
+                               void* stream)
+{
+    int rc = check_tables(t);
+    if (rc) return rc;
+    if ((rc = check_desc(d))) return rc;
+    if (d.rows == 0 || d.groups_per_row == 0) return ECCO_OK;
+    if (!blocks || !y) return ECCO_ERR_ARG;
+    if (!aligned16(blocks) || !aligned16(y)) return ECCO_ERR_ALIGN;
+    return status(launch_decode_act(t, blocks, d, y, (cudaStream_t)stream));
+}
+
 extern "C" int ecco_decode(const ecco_tables* t, const uint8_t* blocks, ecco_desc d, uint16_t* y,
                            void* stream)
 {

@@ -10,6 +10,9 @@
 // hidden by 32 resident warps per SM, and no work is spent on offsets that
 // turn out to be wrong.
 //
+// G = 64 is the activation format (64 values per 512-bit block, the review
+// page's 2x ratio for activations); everything else is shared.
+//
 // Per block: parse the header (scale code, pattern, codebook), form the 16
 // output values bf16(s * C[p][j]) as register byte planes, decode the stream
 // 8 symbols at a time (ecco_block.cuh), write each 16 decoded values with one
@@ -61,7 +64,7 @@ struct DecParams {
 // Each CTA decodes one contiguous, equal share of all blocks of the launch,
 // segment by segment, restaging the segment's tables in shared memory when
 // its share crosses into the next segment.
-template <bool WIDE, int MAXSEG>
+template <bool WIDE, int MAXSEG, int G>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecParams<MAXSEG> P)
 {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         int64_t r = item / gpr, g = item - r * gpr;
         for (; item < end; item += kDecThreads) {
             const uint8_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * ECCO_BLOCK_BYTES;
-            uint16_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * kG;
+            uint16_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * G;
             g += stride_g;
             r += stride_r;
             if (g >= gpr) {
@@ -108,7 +111,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             if (scale_code_is_null(code)) {
                 const uint32_t z[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int k = 0; k < 8; ++k) store16<WIDE>(dst + 16 * k, z, z);
+                for (int k = 0; k < G / 16; ++k) store16<WIDE>(dst + 16 * k, z, z);
                 continue;
             }
             stage_words(ws, kWordStride, q0, q1, q2, q3);
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 
             Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {  // 8 x 16 symbols, one 32-byte store each
+            for (int c = 0; c < G / 16; ++c) {  // 16 symbols, one 32-byte store each
                 uint32_t wa[4], wb[4];
                 chunk_values(st, lut, ws, kWordStride, vp, wa);
                 chunk_values(st, lut, ws, kWordStride, vp, wb);
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 int at = kBlockBits - st.room;
                 for (int k = 0; k < n; ++k, at += kRecBits) {
                     uint32_t rec = read_record(ws, kWordStride, at);
-                    int i = (int)(rec & 127u);
+                    int i = (int)(rec & (uint32_t)(G - 1));  // the 7-bit index, modulo G
                     int qv = (int)(int8_t)(uint8_t)(rec >> 7);
                     float o = __fdiv_rn((float)qv, 127.0f);
                     dst[i] = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
@@ -142,14 +145,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
 }
 
-template <bool WIDE, int MAXSEG>
+template <bool WIDE, int MAXSEG, int G = kG>
 cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
 {
     static int configured = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured != dev) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<WIDE, MAXSEG>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<WIDE, MAXSEG, G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmem);
         if (e != cudaSuccess) return e;
         configured = dev;
@@ -157,7 +160,7 @@ cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
     int64_t want = (P.total + kDecThreads - 1) / kDecThreads;
     int64_t cap = device_sm_count();
     int grid = (int)(want < cap ? want : cap);
-    decode_kernel<WIDE, MAXSEG><<<grid, kDecThreads, kDecSmem, s>>>(P);
+    decode_kernel<WIDE, MAXSEG, G><<<grid, kDecThreads, kDecSmem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -173,6 +176,16 @@ cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecc
     P.total = d.rows * d.groups_per_row;
     P.seg[0] = DecSeg{t->d, blocks, y, d, 0, P.total};
     return wide_ok(y) ? run_decode<true, 1>(P, s) : run_decode<false, 1>(P, s);
+}
+
+cudaError_t launch_decode_act(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
+                              uint16_t* y, cudaStream_t s)
+{
+    DecParams<1> P;
+    P.n_seg = 1;
+    P.total = d.rows * d.groups_per_row;
+    P.seg[0] = DecSeg{t->d, blocks, y, d, 0, P.total};
+    return wide_ok(y) ? run_decode<true, 1, kGAct>(P, s) : run_decode<false, 1, kGAct>(P, s);
 }
 
 // Segments are packed into launches of at most kMultiSeg; empty ones are skipped.

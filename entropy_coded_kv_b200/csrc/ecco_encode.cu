@@ -1,5 +1,6 @@
 // Encoder: 16 lanes per 128-value group (two groups per warp), lane l of a
-// half-warp owning values 8l..8l+7.
+// half-warp owning values 8l..8l+7.  The activation format (G = 64, the review
+// page's 2x ratio for activations) runs the same code with 8 lanes per group.
 //
 // Steps ("Ecco: Improving Memory Bandwidth and Capacity for LLMs via
 // Entropy-aware Cache Compression", review page):
@@ -82,14 +83,17 @@ __device__ __forceinline__ int quantise(const uint32_t* R, float t7, float v)
     return idx;
 }
 
-// Encodes one group with the 16 lanes of `gmask`; hl = lane within the half.
-// cent: centroids [64][16] (SEL = 1 only).
-template <int SEL>
+// Encodes one group of G values with the G/8 lanes of `gmask`; hl = lane
+// within the group.  cent: centroids [64][16] (SEL = 1 only).
+template <int SEL, int G>
 __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, const uint32_t* rows,
-                                             const float* cent, uint32_t* buf, const float2 (&ends)[4],
-                                             const uint16_t* src, uint8_t* dst, int hl, uint32_t gmask,
-                                             int npat, Counters& cnt)
+                                             const float* cent, uint32_t* buf,
+                                             const float2 (&ends)[kNPat / (G / 8)], const uint16_t* src,
+                                             uint8_t* dst, int hl, uint32_t gmask, int npat, Counters& cnt)
 {
+    constexpr int kLanes = G / 8;             // lanes per group
+    constexpr int kPatPerLane = kNPat / kLanes;
+    constexpr int kWords = 16 / kLanes;       // block words each lane stores
     const uint4 q = __ldg(reinterpret_cast<const uint4*>(src) + hl);
     uint32_t b[8] = {q.x & 0xffffu, q.x >> 16, q.y & 0xffffu, q.y >> 16,
                      q.z & 0xffffu, q.z >> 16, q.w & 0xffffu, q.w >> 16};
@@ -121,7 +125,10 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     const uint32_t code = (uint32_t)__ldg(&tb->code_of_mag[key >> 8]) | ((key & 1u) << 7);
     cnt.groups += 1;
     if ((code & 0x7fu) == 0u) {
-        reinterpret_cast<uint32_t*>(dst)[hl] = 0u;
+        if constexpr (kWords == 1)
+            reinterpret_cast<uint32_t*>(dst)[hl] = 0u;
+        else
+            reinterpret_cast<uint2*>(dst)[hl] = make_uint2(0u, 0u);
         cnt.zero += 1;
         return;
     }
@@ -145,14 +152,14 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
         const float umin = hw_minf(gmask, lmin);
         const float umax = hw_maxf(gmask, lmax);
 
-        // ---- pattern: this lane evaluates patterns hl, hl+16, hl+32, hl+48 (those
-        // below npat).  e >= +0, so bit order is value order; a pattern past npat
+        // ---- pattern: this lane evaluates patterns hl + kLanes k (those below
+        // npat).  e >= +0, so bit order is value order; a pattern past npat
         // gets 0xffffffff, above every error including +inf, so a group whose
         // errors are all +inf still gets the lowest index, as scanning does.
         uint32_t eb = 0xffffffffu, bp = 64u;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int pat = hl + 16 * k;
+        for (int k = 0; k < kPatPerLane; ++k) {
+            const int pat = hl + kLanes * k;
             float d0 = __fsub_rn(umin, ends[k].x), d1 = __fsub_rn(umax, ends[k].y);
             float e = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
             const uint32_t ek = (pat < npat) ? __float_as_uint(e) : 0xffffffffu;
@@ -180,7 +187,7 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
             float v = __fadd_rn(__fadd_rn(__fadd_rn(d2[0], d2[1]), __fadd_rn(d2[2], d2[3])),
                                 __fadd_rn(__fadd_rn(d2[4], d2[5]), __fadd_rn(d2[6], d2[7])));
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(gmask, v, o));
+            for (int o = 1; o < kLanes; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(gmask, v, o));
             if (q == 0 || v < best) {
                 best = v;
                 p = q;
@@ -222,10 +229,10 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
         cl[c] = n;
     }
     const int tot = cl[0] + cl[1];
-    int off = tot;  // inclusive scan over the 16 lanes
+    int off = tot;  // inclusive scan over the group's lanes
 #pragma unroll
-    for (int dlt = 1; dlt < 16; dlt <<= 1) {
-        int t = __shfl_up_sync(gmask, off, dlt, 16);
+    for (int dlt = 1; dlt < kLanes; dlt <<= 1) {
+        int t = __shfl_up_sync(gmask, off, dlt, kLanes);
         if (hl >= dlt) off += t;
     }
     off -= tot;
@@ -280,8 +287,14 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     }
 
     __syncwarp(gmask);
-    reinterpret_cast<uint32_t*>(dst)[hl] = buf[hl];
-    buf[hl] = 0u;
+    if constexpr (kWords == 1) {
+        reinterpret_cast<uint32_t*>(dst)[hl] = buf[hl];
+        buf[hl] = 0u;
+    } else {
+        reinterpret_cast<uint2*>(dst)[hl] = make_uint2(buf[2 * hl], buf[2 * hl + 1]);
+        buf[2 * hl] = 0u;
+        buf[2 * hl + 1] = 0u;
+    }
     __syncwarp(gmask);
 }
 
@@ -304,17 +317,18 @@ struct EncParams {  // by value: no device-side segment table
 
 // Each CTA encodes one contiguous, equal share of all groups of the launch,
 // segment by segment, restaging the pattern rows when it enters a new segment.
-template <int MAXSEG, int SEL>
+template <int MAXSEG, int SEL, int G>
 __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_constant__ EncParams<MAXSEG> P)
 {
+    constexpr int kLanes = G / 8, kGpw = 32 / kLanes;  // lanes per group, groups per warp
     __shared__ uint32_t rows[kNPat * kRow];
     __shared__ float cent[SEL ? kNPat * 16 : 1];  // C[p][j] pattern-major (full-MSE selection)
-    __shared__ uint32_t bufs[2 * kEncWarps][20];
+    __shared__ uint32_t bufs[kGpw * kEncWarps][20];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int i = tid; i < 2 * kEncWarps * 20; i += blockDim.x) (&bufs[0][0])[i] = 0u;
-    const int half = lane >> 4, hl = lane & 15;
-    const uint32_t gmask = 0xffffu << (16 * half);
-    uint32_t* buf = bufs[2 * warp + half];
+    for (int i = tid; i < kGpw * kEncWarps * 20; i += blockDim.x) (&bufs[0][0])[i] = 0u;
+    const int sub = lane / kLanes, hl = lane % kLanes;
+    const uint32_t gmask = (uint32_t)((1ull << kLanes) - 1ull) << (kLanes * sub);
+    uint32_t* buf = bufs[kGpw * warp + sub];
     Counters cnt = {0, 0, 0, 0, 0, 0, 0ull};
 
     const int64_t share = (P.total + gridDim.x - 1) / gridDim.x;
@@ -353,21 +367,21 @@ __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_
         if constexpr (SEL == 1) {
             for (int i = tid; i < kNPat * 16; i += blockDim.x) cent[i] = tb->Ct[i & 15][i >> 4];
         }
-        float2 ends[4];
+        float2 ends[kNPat / kLanes];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) ends[k] = __ldg(&tb->ends[hl + 16 * k]);
+        for (int k = 0; k < kNPat / kLanes; ++k) ends[k] = __ldg(&tb->ends[hl + kLanes * k]);
         __syncthreads();
 
-        constexpr int kPerRound = 2 * kEncWarps;  // groups per CTA round
+        constexpr int kPerRound = kGpw * kEncWarps;  // groups per CTA round
         const int64_t gpr = S.d.groups_per_row;
         const int64_t stride_r = kPerRound / gpr, stride_g = kPerRound % gpr;
-        int64_t item = lo - S.begin + 2 * warp + half;
+        int64_t item = lo - S.begin + kGpw * warp + sub;
         const int64_t end = stop - S.begin;
         int64_t r = item / gpr, g = item - r * gpr;
         for (; item < end; item += kPerRound) {
-            const uint16_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * kG;
+            const uint16_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * G;
             uint8_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * ECCO_BLOCK_BYTES;
-            encode_group<SEL>(tb, rows, cent, buf, ends, src, dst, hl, gmask, P.npat, cnt);
+            encode_group<SEL, G>(tb, rows, cent, buf, ends, src, dst, hl, gmask, P.npat, cnt);
             g += stride_g;
             r += stride_r;
             if (g >= gpr) {
@@ -389,17 +403,17 @@ __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_
     }
 }
 
-template <int MAXSEG>
+template <int MAXSEG, int G = kG>
 cudaError_t run_encode(const EncParams<MAXSEG>& P, int select, cudaStream_t s)
 {
-    const int per_cta = 2 * kEncWarps;
+    const int per_cta = (32 / (G / 8)) * kEncWarps;
     int64_t want = (P.total + per_cta - 1) / per_cta;
     int64_t cap = (int64_t)device_sm_count() * 3;  // resident CTAs at 3 per SM
     int grid = (int)(want < cap ? want : cap);
     if (select == ECCO_SELECT_MSE)
-        encode_kernel<MAXSEG, 1><<<grid, kEncWarps * 32, 0, s>>>(P);
+        encode_kernel<MAXSEG, 1, G><<<grid, kEncWarps * 32, 0, s>>>(P);
     else
-        encode_kernel<MAXSEG, 0><<<grid, kEncWarps * 32, 0, s>>>(P);
+        encode_kernel<MAXSEG, 0, G><<<grid, kEncWarps * 32, 0, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -415,6 +429,18 @@ cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_de
     P.stats = stats;
     P.seg[0] = EncSeg{t->d, x, blocks, d, 0, P.total};
     return run_encode<1>(P, select, s);
+}
+
+cudaError_t launch_encode_act(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
+                              uint8_t* blocks, ecco_stats* stats, cudaStream_t s)
+{
+    EncParams<1> P;
+    P.n_seg = 1;
+    P.npat = kNPat;
+    P.total = d.rows * d.groups_per_row;
+    P.stats = stats;
+    P.seg[0] = EncSeg{t->d, x, blocks, d, 0, P.total};
+    return run_encode<1, kGAct>(P, ECCO_SELECT_MINMAX, s);
 }
 
 // Segments are packed into launches of at most kMultiSeg; empty ones are skipped.

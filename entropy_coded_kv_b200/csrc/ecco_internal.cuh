@@ -17,6 +17,7 @@
 namespace ecco {
 
 constexpr int kG = 128;           // values per group
+constexpr int kGAct = 64;         // values per group, activation format (2x)
 constexpr int kNPat = 64;         // shared patterns per tensor
 constexpr int kNCent = 15;        // centroids per pattern
 constexpr int kNBook = 4;         // codebooks per pattern
@@ -70,6 +71,11 @@ cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t row
 cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                            const uint16_t* x, int batch, float* y, cudaStream_t s);
 cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s);
+// Activation format: 64-value groups (the descriptor counts 64-value groups).
+cudaError_t launch_encode_act(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
+                              uint8_t* blocks, ecco_stats* stats, cudaStream_t s);
+cudaError_t launch_decode_act(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
+                              uint16_t* y, cudaStream_t s);
 cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats,
                                 cudaStream_t s);
 

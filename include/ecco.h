@@ -142,6 +142,22 @@ int ecco_select_encode_ex(const ecco_tables* tables, const uint16_t* x_bf16, ecc
                           uint8_t* blocks, ecco_stats* dev_stats, int select, int n_patterns,
                           void* stream);
 
+/* Activation format (free parameters: "Group size for activations = 64" and
+ * the 2x compression target for activations; Fig. 9 text: the low compression
+ * ratio compressor reuses the high-ratio compressor's components): every
+ * 64-value bf16 group becomes one 64-byte block with the same header, symbols,
+ * codebook choice, clipping and padding rules as above (records keep the
+ * 15-bit layout with an index below 64; the decoder takes the 7-bit index
+ * modulo 64).  Here a descriptor's group index addresses 64 bf16 values
+ * (128 bytes) on the bf16 side.  Tables use the same blob layout, learned on
+ * 64-value groups.  Alignment, errors and stats as ecco_select_encode /
+ * ecco_decode. */
+#define ECCO_GROUP_ACT 64
+int ecco_select_encode_act(const ecco_tables* tables, const uint16_t* x_bf16, ecco_desc desc,
+                           uint8_t* blocks, ecco_stats* dev_stats, void* stream);
+int ecco_decode_act(const ecco_tables* tables, const uint8_t* blocks, ecco_desc desc, uint16_t* y_bf16,
+                    void* stream);
+
 /* Decoder (the review page's decompressor, Fig. 8 caption): every block of
  * `blocks` described by `desc` becomes 128 bf16 values in `y_bf16`.  Any
  * 64-byte pattern decodes deterministically (malformed blocks included).

@@ -121,16 +121,19 @@ def test_decode_garbage_blocks_bit_exact(tname):
     np.testing.assert_array_equal(bits(y).reshape(-1, 128), oracle.decode(blob, blocks, nthreads=8))
 
 
-def test_golden_blocks_on_gpu():
+@pytest.mark.parametrize("gs", [128, 64])
+def test_golden_blocks_on_gpu(gs):
     import test_oracle_pins as P
     blob, spec = P.golden_tables()
     t = ecco.Tables(blob, DEV)
-    xs = np.stack([P.expand(c["x"]) for c in spec["cases"]])
-    want = np.stack([P.assemble_stream(c["stream"]) for c in spec["cases"]])
-    got = ecco.encode(to_dev_bf16(xs), t).cpu().numpy()
+    cases = [c for c in spec["cases"] if c.get("group", 128) == gs]
+    enc, dec = (ecco.encode, ecco.decode) if gs == 128 else (ecco.encode_act, ecco.decode_act)
+    xs = np.stack([P.expand(c["x"], gs) for c in cases])
+    want = np.stack([P.assemble_stream(c["stream"]) for c in cases])
+    got = enc(to_dev_bf16(xs), t).cpu().numpy()
     np.testing.assert_array_equal(got, want)
-    y = ecco.decode(torch.from_numpy(want).to(DEV), t)
-    np.testing.assert_array_equal(bits(y).reshape(-1, 128), np.stack([P.expand(c["decoded"]) for c in spec["cases"]]))
+    y = dec(torch.from_numpy(want).to(DEV), t)
+    np.testing.assert_array_equal(bits(y).reshape(-1, gs), np.stack([P.expand(c["decoded"], gs) for c in cases]))
 
 
 @pytest.mark.parametrize("n", [1, 2, 31, 32, 33, 255, 257, 1023, 1025, 148 * 1024 + 5])

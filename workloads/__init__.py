@@ -183,6 +183,19 @@ def c5_calibration(layer: int, device="cpu", seed: int = 105):
     return kv_cache((1, 8, 4096, 128), seed * 1000 + layer, device)
 
 
+def hidden_states(tokens: int, hidden: int = 4096, seed: int = 6, device="cpu", n_outlier_ch: int = 8,
+                  outlier_mult: float = 20.0, sigma: float = 0.5) -> torch.Tensor:
+    """Activations [tokens, hidden] bf16 for the 64-value-group format: N(0,1)
+    times a per-channel LogNormal(0, sigma) scale, n_outlier_ch channels
+    multiplied by outlier_mult (the channel-outlier shape of LLM activations)."""
+    g = _gen(seed, device)
+    scale = torch.exp(torch.randn(hidden, generator=g, device=device) * sigma)
+    ch = torch.randperm(hidden, generator=g, device=device)[:n_outlier_ch]
+    scale[ch] *= outlier_mult
+    z = torch.randn(tokens, hidden, generator=g, device=device, dtype=torch.float32)
+    return (z * scale.view(1, hidden)).to(torch.bfloat16)
+
+
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 bit patterns (host copy)."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
