@@ -25,7 +25,7 @@ BLOCK_BYTES = 64
 
 __all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
            "decode_attention", "attention_workspace_bytes", "decode_attention_static",
-           "encode_act", "decode_act", "GROUP_ACT",
+           "encode_act", "decode_act", "GROUP_ACT", "learn_tables", "huffman_lengths",
            "new_stats", "read_stats", "flat_desc", "kv_append_desc", "EccoError", "Desc"]
 
 
@@ -263,6 +263,33 @@ def decode_act(blocks: torch.Tensor, tables: Tables, out: torch.Tensor | None = 
     rc = _lib.load().ecco_decode_act(tables.handle, ctypes.c_void_p(blocks.data_ptr()), desc,
                                      ctypes.c_void_p(out.data_ptr()), _stream(blocks.device))
     _lib.check(rc, "ecco_decode_act")
+    return out
+
+
+def learn_tables(sample: torch.Tensor, seed: int = 0, n_patterns: int = 64, group: int = GROUP) -> bytes:
+    """Table blob learned on the GPU (ecco_learn_tables) from a bf16 device
+    tensor whose numel is a multiple of `group` (128, or 64 for activations)."""
+    if not isinstance(sample, torch.Tensor) or sample.dtype != torch.bfloat16 or sample.device.type != "cuda":
+        raise TypeError("sample must be a bf16 CUDA tensor")
+    x = sample.contiguous()
+    if x.numel() % group:
+        raise ValueError(f"sample.numel() must be a multiple of {group}")
+    blob = ctypes.create_string_buffer(_lib.TABLES_BYTES)
+    with torch.cuda.device(x.device):
+        rc = _lib.load().ecco_learn_tables(ctypes.c_void_p(x.data_ptr()), x.numel() // group, group, n_patterns,
+                                           int(seed) & (2 ** 64 - 1), blob, _lib.TABLES_BYTES, _stream(x.device))
+    _lib.check(rc, "ecco_learn_tables")
+    return blob.raw
+
+
+def huffman_lengths(weights, max_len: int = 8):
+    """Optimal length-limited prefix-code lengths (package-merge, host)."""
+    import numpy as np
+    w = np.ascontiguousarray(np.asarray(weights, dtype=np.float64))
+    out = np.zeros(w.size, dtype=np.uint8)
+    rc = _lib.load().ecco_huffman_lengths(ctypes.c_void_p(w.ctypes.data), w.size, max_len,
+                                          ctypes.c_void_p(out.ctypes.data))
+    _lib.check(rc, "ecco_huffman_lengths")
     return out
 
 

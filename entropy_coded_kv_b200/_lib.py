@@ -27,7 +27,7 @@ EXPORTED = [
     "ecco_decode_gemv", "ecco_decode_multi", "ecco_encode_multi", "ecco_strerror",
     "ecco_abi_version", "ecco_device_timeouts", "ecco_decode_attention",
     "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static", "ecco_select_encode_ex",
-    "ecco_select_encode_act", "ecco_decode_act",
+    "ecco_select_encode_act", "ecco_decode_act", "ecco_learn_tables", "ecco_huffman_lengths",
 ]
 
 
@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_decode.argtypes = [P, P, Desc, P, P]
     L.ecco_select_encode_ex.argtypes = [P, P, Desc, P, P, I, I, P]
     L.ecco_select_encode_act.argtypes = [P, P, Desc, P, P, P]
+    L.ecco_learn_tables.argtypes = [P, I64, I, I, ctypes.c_uint64, P, ctypes.c_size_t, P]
+    L.ecco_huffman_lengths.argtypes = [P, I, I, P]
     L.ecco_decode_act.argtypes = [P, P, Desc, P, P]
     L.ecco_decode_gemv.argtypes = [P, P, I64, I64, P, I, P, P]
     L.ecco_decode_multi.argtypes = [ctypes.POINTER(Segment), I, P]

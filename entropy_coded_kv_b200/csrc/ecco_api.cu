@@ -1,5 +1,6 @@
 // C ABI entry points: argument validation, device checks, dispatch to the
 // kernel launchers.  Nothing here allocates device memory.
+#include <cmath>
 #include <cstdint>
 
 #include "ecco_internal.cuh"
@@ -194,6 +195,32 @@ extern "C" int ecco_decode_attention(const ecco_tables* kt, const ecco_tables* v
         return ECCO_ERR_ALIGN;
     return status(launch_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, scale,
                                    out, static_cast<float*>(ws), (cudaStream_t)stream));
+}
+
+extern "C" int ecco_learn_tables(const uint16_t* x, int64_t n_groups, int group, int n_patterns, uint64_t seed,
+                                 void* blob, size_t blob_bytes, void* stream)
+{
+    if (!x || !blob || blob_bytes < ECCO_TABLES_BYTES) return ECCO_ERR_ARG;
+    if (n_groups < 1 || n_groups > ((int64_t)1 << 34)) return ECCO_ERR_ARG;
+    if (group != ECCO_GROUP && group != ECCO_GROUP_ACT) return ECCO_ERR_ARG;
+    if (n_patterns < 1 || n_patterns > ECCO_NPAT) return ECCO_ERR_ARG;
+    if (!aligned16(x)) return ECCO_ERR_ALIGN;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ECCO_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ECCO_ERR_CUDA;
+    if (prop.major != 10) return ECCO_ERR_UNSUPPORTED;
+    return status(learn_tables(x, n_groups, group, n_patterns, seed, static_cast<uint8_t*>(blob),
+                               (cudaStream_t)stream));
+}
+
+extern "C" int ecco_huffman_lengths(const double* w, int n, int max_len, uint8_t* lens)
+{
+    if (!w || !lens || n < 1 || max_len < 1 || max_len > 30) return ECCO_ERR_ARG;
+    if (n > 1 && (int64_t)n > ((int64_t)1 << max_len)) return ECCO_ERR_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!(w[i] > 0.0) || !std::isfinite(w[i])) return ECCO_ERR_ARG;
+    return huffman_lengths(w, n, max_len, lens) == 0 ? ECCO_OK : ECCO_ERR_ARG;
 }
 
 extern "C" const char* ecco_strerror(int code)

@@ -85,6 +85,11 @@ cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const
                              const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
                              const uint16_t* q, float scale, float* out, float* ws, cudaStream_t s);
 
+// Table learner (offline): the blob of one tensor from a device bf16 sample.
+cudaError_t learn_tables(const uint16_t* x, int64_t n_groups, int G, int npat, uint64_t seed, uint8_t* blob,
+                         cudaStream_t s);
+int huffman_lengths(const double* w, int n, int max_len, uint8_t* lens);
+
 int device_sm_count();
 
 // ------------------------------------------------------------ device helpers

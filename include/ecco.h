@@ -242,6 +242,32 @@ int ecco_decode_attention_static(const ecco_tables* k_tables, const ecco_tables*
                                  int batch, int kv_heads, int group, int seq_len, const uint16_t* q_bf16,
                                  float scale, float* out, void* stream);
 
+/* Table learner on the GPU (offline; blocking; allocates and frees its own
+ * temporaries; not for the hot path).  Learns one tensor's table blob -- the
+ * per-tensor parameters the review page says are learned once, offline ("What
+ * carries the argument"; free parameters S = 64, H = 4, 15 centroids; referee
+ * comment 1: lengths <= 8) -- from `n_groups` groups of `group` (128, or 64
+ * for the activation format) bf16 values at `sample_bf16` (device, 16-byte
+ * aligned):
+ *   S_t = absmax / 448; each of up to 16,384 sampled groups (seeded sample) is
+ *   scaled by its FP8 group scale, its largest element set aside and the rest,
+ *   sorted, summarised by 15 equal-count bin means; k-means++ / Lloyd (20
+ *   iterations) over those gives the patterns; 4 rounds move every centroid to
+ *   the mean of the values the encoder's own rules (min/max pattern,
+ *   thresholds) give it; per pattern, 4 codebooks from clustered symbol
+ *   histograms, each an optimal prefix code with lengths <= 8 (package-merge).
+ * `n_patterns` < 64 learns that many (rows past it repeat row 0; encode with
+ * ecco_select_encode_ex and the same count).  The blob (ECCO_TABLES_BYTES,
+ * host memory) is the same for the same sample and seed. */
+int ecco_learn_tables(const uint16_t* sample_bf16, int64_t n_groups, int group, int n_patterns,
+                      uint64_t seed, void* blob_out, size_t blob_bytes, void* stream);
+
+/* Optimal prefix-code lengths for n symbols of the given (positive) weights,
+ * every length <= max_len (package-merge; ties in symbol order).  Host only,
+ * no device needed.  Returns ECCO_ERR_ARG if n < 1, max_len < 1 or
+ * n > 2^max_len. */
+int ecco_huffman_lengths(const double* weights, int n, int max_len, uint8_t* lengths_out);
+
 /* Number of bounded device-side waits (tensor-core decode+GEMV pipeline) that
  * gave up since the library was loaded on the current device; 0 in normal
  * operation.  A kernel whose wait gives up skips the rest of its work instead
