@@ -378,35 +378,6 @@ class MLPWorkload(Workload):
                 "bytes": 2 * n * 256, "what": f"encode {n} groups + decode {n} blocks (1/{round(1 / frac)} of a step, GEMV not sampled)"}
 
 
-def _learn_many(samples, seed=0):
-    """Learns one table blob per sample (uint16 bf16 bits [n, 128]) in a
-    spawn-context process pool (workers hold no CUDA state)."""
-    import multiprocessing as mp
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(min(len(samples), max(1, (os.cpu_count() or 2) - 1))) as pool:
-        return pool.starmap(_learn_one, [(s, seed) for s in samples])
-
-
-def _learn_one(bits, seed):
-    import numpy as np
-    import torch
-    sys.path.insert(0, ROOT)
-    from entropy_coded_kv_b200.calib import learn_tables
-    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-    return learn_tables(t, seed=seed, max_groups=8192)
-
-
-def _sample_groups(t, k, seed):
-    """k groups of a device tensor, chosen by a seeded permutation, as host bits."""
-    import torch
-    import workloads as W
-    n = t.numel() // 128
-    g = torch.Generator(device=t.device)
-    g.manual_seed(seed)
-    idx = torch.randperm(n, generator=g, device=t.device)[: min(k, n)]
-    return W.bf16_bits(t.view(n, 128)[idx])
-
-
 class ModelWorkload(Workload):
     """All 224 weight tensors of a 32-layer Llama-3-8B-shaped model: encode the
     whole set, decode the whole set (one multi-segment launch per 64 tensors)."""
@@ -419,13 +390,12 @@ class ModelWorkload(Workload):
         self.torch, self.ecco, self.dev = torch, ecco, dev
         self.desc = ("Llama-3-8B-shaped weights, 32 layers x {q,k,v,o 4096/1024 x 4096; gate,up 14336 x 4096; "
                      "down 4096 x 14336}, Student-t(5) x 0.02, per-tensor tables: whole-model encode + decode")
-        self.w, samples = [], []
+        self.w, self.tables = [], []
         for layer in range(W.C4_LAYERS):
             for name, _, _ in W.C4_SHAPES:
                 t = W.c4_tensor(layer, name, device=dev, seed=4 + seed_offset)
                 self.w.append(t)
-                samples.append(_sample_groups(t, 8192, seed=layer))
-        self.tables = [ecco.Tables(b, dev) for b in _learn_many(samples)]
+                self.tables.append(ecco.Tables(ecco.learn_tables(t, seed=layer), dev))  # GPU learner
         self.blocks = [torch.empty((t.numel() // 128, 64), dtype=torch.uint8, device=dev) for t in self.w]
         self.out = [torch.empty_like(t) for t in self.w]
         self.n = sum(t.numel() // 128 for t in self.w)
@@ -497,14 +467,13 @@ class LongCtxWorkload(Workload):
         self.desc = ("long-context KV cache, 32 layers x K,V x [1, 8, 131072, 128] bf16 (17.2 GB), per-layer K/V "
                      "tables from [1, 8, 4096, 128] calibration samples: decode the whole cache + append one token "
                      "per layer (512 groups)")
-        self.caches, samples = [], []
+        self.caches, self.tables = [], []
         for layer in range(32):
             K, V = W.c5_layer(layer, device=dev, seed=5 + seed_offset)
             Kc, Vc = W.c5_calibration(layer, device=dev, seed=105 + seed_offset)
             self.caches += [K, V]
-            samples += [W.bf16_bits(Kc.reshape(-1, 128)), W.bf16_bits(Vc.reshape(-1, 128))]
+            self.tables += [ecco.Tables(ecco.learn_tables(c, seed=layer), dev) for c in (Kc, Vc)]  # GPU learner
             del Kc, Vc
-        self.tables = [ecco.Tables(b, dev) for b in _learn_many(samples)]
         self.blocks = [torch.empty((c.numel() // 128, 64), dtype=torch.uint8, device=dev) for c in self.caches]
         ecco.encode_multi([ecco.Seg(tb, c, b) for tb, c, b in zip(self.tables, self.caches, self.blocks)])
         self.out = [torch.empty_like(c) for c in self.caches]
