@@ -961,27 +961,40 @@ def main():
         dist.destroy_process_group()
 
 
-def source_hash() -> str:
-    import glob
+# Sources each profiled kernel is built from: its DRAM traffic in
+# profiles/traffic.json is used only while these files are unchanged.
+KERNEL_SOURCES = {
+    "decode_kernel": ["ecco_decode.cu", "ecco_block.cuh"],
+    "decode_kernel<G=64>": ["ecco_decode.cu", "ecco_block.cuh"],
+    "encode_kernel<.,SEL=1>": ["ecco_encode.cu"],
+    "attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_block.cuh"],
+}
+
+
+def source_hash(files) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "entropy_coded_kv_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for f in files:
+        with open(os.path.join(ROOT, "entropy_coded_kv_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(workload, kernel):
-    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
-    or None when no capture matches or the kernel sources changed since."""
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/traffic.json), or None when no capture matches or the
+    kernel's sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f)
-    if d.get("source_hash") != source_hash():
+        entry = json.load(f).get("entries", {}).get(f"{workload}:{kernel}")
+    if not entry:
         return None
-    return d.get(f"{workload}:{kernel.split()[0]}")
+    files = KERNEL_SOURCES.get(kernel.split(" ")[0], [])
+    if not files or entry.get("source_hash") != source_hash(files):
+        return None
+    return entry.get("dram_bytes_per_launch")
 
 
 def run_reference(args, world):
