@@ -104,6 +104,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 g -= gpr;
                 r += 1;
             }
+            if (item + kDecThreads < end)  // this thread's next block: on its way to L2 while this one decodes
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(S.src + (S.d.src_offset + r * S.d.src_row_stride + g) *
+                                                                            ECCO_BLOCK_BYTES));
 
             uint4 q0 = ldg_nc_v4(src), q1 = ldg_nc_v4(src + 16), q2 = ldg_nc_v4(src + 32),
                   q3 = ldg_nc_v4(src + 48);
