@@ -89,13 +89,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         __syncthreads();
 
         // local group index within the segment; consecutive threads take
-        // consecutive groups, kDecThreads per round
+        // consecutive groups.  The CTA's part of the segment is spread evenly
+        // over the fewest rounds of at most kDecThreads (4 rounds of 886 rather
+        // than 3 of 1024 and one of 470), so no round runs the SM half empty.
         const int64_t gpr = S.d.groups_per_row;
-        const int64_t stride_r = kDecThreads / gpr, stride_g = kDecThreads % gpr;
+        const int64_t part = stop - lo;
+        const int64_t rounds = (part + kDecThreads - 1) / kDecThreads;
+        const int64_t per_round = (part + rounds - 1) / rounds;
+        const int64_t stride_r = per_round / gpr, stride_g = per_round % gpr;
         int64_t item = lo - S.begin + tid;
-        const int64_t end = stop - S.begin;
+        const int64_t end = (tid < per_round) ? stop - S.begin : 0;
         int64_t r = item / gpr, g = item - r * gpr;
-        for (; item < end; item += kDecThreads) {
+        for (; item < end; item += per_round) {
             const uint8_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * ECCO_BLOCK_BYTES;
             uint16_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * G;
             g += stride_g;
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 g -= gpr;
                 r += 1;
             }
-            if (item + kDecThreads < end)  // this thread's next block: on its way to L2 while this one decodes
+            if (item + per_round < end)  // this thread's next block: on its way to L2 while this one decodes
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(S.src + (S.d.src_offset + r * S.d.src_row_stride + g) *
                                                                             ECCO_BLOCK_BYTES));
 
