@@ -5,76 +5,101 @@
 // memory (the review page's figure list: "Normalized Memory Requests for a
 // GEMM Kernel" -- compressed weights are what crosses the memory bus).
 //
-// Layout of the work: a warp owns 32 consecutive rows and walks a range of
-// column groups in lockstep, so at every step all lanes need the same x[k]
-// (a broadcast shared-memory read).  Each lane decodes its row's block
-// serially (one lookup per symbol, as in the decoder) and multiplies every
-// decoded bf16 value, exactly, in fp32 against the batch of x.  An outlier
-// record replaces the value of its element, so its contribution is corrected
-// by (new - old) * x, with the old symbol kept in shared memory.  Partial row
-// sums of the column ranges are combined with fp32 atomics.
+// Layout of the work: a unit is one row per thread (1024 rows at batch 1, 512
+// at batch 2..4) x one column group; a CTA owns a balanced, contiguous range of units in (row tile, column
+// group) order and stays resident (one CTA per SM), so every SM gets the same
+// amount of work instead of a grid of whole tiles that leaves part of the last
+// wave idle.  A warp owns 32 consecutive rows, so at every step all lanes need
+// the same x[k] (a broadcast shared-memory read); x is staged in windows of 32
+// column groups.  Each lane decodes its row's block serially (one lookup per
+// symbol, as in the decoder) and multiplies every decoded bf16 value, exactly,
+// in fp32 against the batch of x.  An outlier record replaces the value of its
+// element, so its contribution is corrected by (new - old) * x, with the old
+// symbol kept in shared memory.  A thread's row sum is added to y (fp32
+// atomics) when its unit range moves to the next row tile and at the end.
 #include "ecco_block.cuh"
 
 namespace ecco {
 namespace {
 
-constexpr int kGvThreads = 512;
-constexpr int kGvWarps = kGvThreads / 32;
-constexpr int kGvColGroups = 4;   // column groups per CTA (x slice of 512 values)
-constexpr int kGvStride = kGvThreads;
-
+constexpr int kGvWin = 32;        // column groups of x staged at a time (4096 values)
 constexpr size_t kGvLut = 65536;
 constexpr size_t kGvCt = 4096;
-constexpr size_t kGvWords = 16 * kGvStride * 4;
-constexpr size_t kGvNib = 16 * kGvThreads * 4;
+
+// Threads per CTA (= rows per unit): batch 1 fits the decoder's 1024 threads
+// (64 registers); larger batches need more registers for the accumulators.
+template <int B>
+constexpr int gv_threads()
+{
+    return B == 1 ? 1024 : 512;
+}
 
 template <int B>
 constexpr size_t gv_smem()
 {
-    return kGvLut + kGvCt + kGvWords + kGvNib + (size_t)kGvColGroups * kG * B * 4;
+    return kGvLut + kGvCt + (size_t)16 * gv_threads<B>() * 4 * 2 + (size_t)kGvWin * kG * B * 4;
 }
 
 template <int B>
-__global__ void __launch_bounds__(kGvThreads, 1)
+__global__ void __launch_bounds__(gv_threads<B>(), 1)
     gemv_kernel(const DevTables* __restrict__ tb, const uint8_t* __restrict__ blocks, int64_t rows,
                 int64_t gpr, const uint16_t* __restrict__ x, int batch, int64_t cols,
                 float* __restrict__ y)
 {
+    constexpr int kGvThreads = gv_threads<B>(), kGvStride = kGvThreads;
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kGvLut);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kGvLut + kGvCt);
     uint32_t* s_nib = s_w + 16 * kGvStride;
-    float* s_x = reinterpret_cast<float*>(s_nib + 16 * kGvThreads);  // [k][B]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float* s_x = reinterpret_cast<float*>(s_nib + 16 * kGvThreads);  // [k][B], one window
+    const int tid = threadIdx.x;
 
-    const int64_t g0 = (int64_t)blockIdx.y * kGvColGroups;
-    const int ng = (int)min((int64_t)kGvColGroups, gpr - g0);
-    {
-        stage_tables<kGvThreads>(tb, s_lut, s_Ct, tid);
-        for (int i = tid; i < kGvColGroups * kG * B; i += kGvThreads) {
-            int k = i / B, bb = i - k * B;
-            float v = 0.0f;
-            if (bb < batch && k < ng * kG) v = bf16_bits_to_f32(x[(int64_t)bb * cols + g0 * kG + k]);
-            s_x[i] = v;
-        }
-    }
+    stage_tables<kGvThreads>(tb, s_lut, s_Ct, tid);
     const float S_t = tb->S_t;
-    __syncthreads();
+    const int64_t tiles = (rows + kGvThreads - 1) / kGvThreads;
+    const int64_t units = tiles * gpr;
+    const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
 
-    const int64_t row = ((int64_t)blockIdx.x * kGvWarps + warp) * 32 + lane;
-    const bool row_ok = row < rows;
     uint32_t* ws = s_w + tid;
     uint32_t* nibs = s_nib + tid;
     float acc[B];
 #pragma unroll
     for (int bb = 0; bb < B; ++bb) acc[bb] = 0.0f;
+    int64_t cur_tile = u0 / gpr, cur_win = -1;
 
-    for (int gi = 0; gi < ng; ++gi) {
-        const float* xs = s_x + gi * kG * B;
+    for (int64_t u = u0; u < u1; ++u) {
+        const int64_t tile = u / gpr, gcol = u - tile * gpr;
+        if (tile != cur_tile) {  // this thread's row changes: add its sum to y
+            const int64_t prow = cur_tile * kGvThreads + tid;
+            if (prow < rows) {
+#pragma unroll
+                for (int bb = 0; bb < B; ++bb)
+                    if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + prow], acc[bb]);
+            }
+#pragma unroll
+            for (int bb = 0; bb < B; ++bb) acc[bb] = 0.0f;
+            cur_tile = tile;
+        }
+        const int64_t win = gcol / kGvWin;
+        if (win != cur_win) {  // uniform across the CTA
+            __syncthreads();   // the previous window is no longer read (and the tables are staged)
+            const int64_t k0 = win * kGvWin * kG;
+            const int nk = (int)min((int64_t)kGvWin * kG, cols - k0);
+            for (int i = tid; i < kGvWin * kG * B; i += kGvThreads) {
+                const int k = i / B, bb = i - k * B;
+                s_x[i] = (bb < batch && k < nk) ? bf16_bits_to_f32(x[(int64_t)bb * cols + k0 + k]) : 0.0f;
+            }
+            __syncthreads();
+            cur_win = win;
+        }
+        const int64_t row = tile * kGvThreads + tid;
+        const bool row_ok = row < rows;
+        const float* xs = s_x + (gcol - win * kGvWin) * kG * B;
+        {
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, q2 = q0, q3 = q0;
         if (row_ok) {
-            const uint8_t* src = blocks + (row * gpr + g0 + gi) * ECCO_BLOCK_BYTES;
+            const uint8_t* src = blocks + (row * gpr + gcol) * ECCO_BLOCK_BYTES;
             q0 = ldg_nc_v4(src);
             q1 = ldg_nc_v4(src + 16);
             q2 = ldg_nc_v4(src + 32);
@@ -123,11 +148,13 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                 for (int bb = 0; bb < B; ++bb) acc[bb] = fmaf(dv, xi[bb], acc[bb]);
             }
         }
+        }
     }
-    if (row_ok) {
+    const int64_t prow = cur_tile * kGvThreads + tid;
+    if (u1 > u0 && prow < rows) {
 #pragma unroll
         for (int bb = 0; bb < B; ++bb)
-            if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + row], acc[bb]);
+            if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + prow], acc[bb]);
     }
 }
 
@@ -145,9 +172,9 @@ cudaError_t run_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, 
     cudaError_t e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)batch * (size_t)rows, s);
     if (e != cudaSuccess) return e;
     const int64_t gpr = cols / kG;
-    dim3 grid((unsigned)((rows + kGvThreads - 1) / kGvThreads),
-              (unsigned)((gpr + kGvColGroups - 1) / kGvColGroups));
-    gemv_kernel<B><<<grid, kGvThreads, gv_smem<B>(), s>>>(t->d, blocks, rows, gpr, x, batch, cols, y);
+    const int64_t units = (rows + gv_threads<B>() - 1) / gv_threads<B>() * gpr;
+    const int grid = (int)(units < device_sm_count() ? units : device_sm_count());  // one resident CTA per SM
+    gemv_kernel<B><<<grid, gv_threads<B>(), gv_smem<B>(), s>>>(t->d, blocks, rows, gpr, x, batch, cols, y);
     return cudaGetLastError();
 }
 
