@@ -850,8 +850,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        dist.init_process_group("nccl" if args.impl == "ecco" else "gloo",
-                                timeout=datetime.timedelta(seconds=300))
+        if args.impl == "ecco":  # one GPU per rank, bound before the first collective
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
 
     if args.impl == "reference":
         if rank == 0:

@@ -393,3 +393,26 @@ def test_no_device_wait_gave_up():
     n = ctypes.c_uint(123)
     assert _lib.load().ecco_device_timeouts(ctypes.byref(n)) == 0
     assert n.value == 0
+
+
+def test_offsets_past_4_gib():
+    """Descriptors that address groups more than 2^32 bytes into the buffers
+    (row stride 2^25 groups = 8 GiB of bf16): every index is 64-bit."""
+    blob = table_set("learned_kv")
+    t = ecco.Tables(blob, DEV)
+    gpr, stride = 300, 1 << 25
+    xb = inputs("kv", 2 * gpr, seed=77)
+    src = torch.empty((stride + gpr, 128), dtype=torch.bfloat16, device=DEV)  # ~8.6 GB, not written
+    src[:gpr] = to_dev_bf16(xb[: gpr * 128]).view(gpr, 128)
+    src[stride:] = to_dev_bf16(xb[gpr * 128:]).view(gpr, 128)
+    blocks = torch.empty((2 * gpr, 64), dtype=torch.uint8, device=DEV)
+    ecco.encode(src, t, out=blocks, desc=_lib.Desc(2, gpr, stride, gpr, 0, 0))
+    want, _ = oracle.encode(blob, xb, nthreads=8)
+    np.testing.assert_array_equal(blocks.cpu().numpy(), want)
+    out = torch.empty_like(src)
+    ecco.decode(blocks, t, out=out, desc=_lib.Desc(2, gpr, gpr, stride, 0, 0))
+    wy = oracle.decode(blob, want, nthreads=8)
+    np.testing.assert_array_equal(bits(out[:gpr]).reshape(-1, 128), wy[:gpr])
+    np.testing.assert_array_equal(bits(out[stride:]).reshape(-1, 128), wy[gpr:])
+    del src, out
+    torch.cuda.empty_cache()
