@@ -74,6 +74,24 @@ __device__ __forceinline__ uint32_t keyof(uint32_t v, int i)
     return ((v & 0x7fffu) << 8) | ((uint32_t)(127 - i) << 1) | (v >> 15);
 }
 
+// Sorts 8 keys descending (Batcher's odd-even merge sort, 19 comparators).
+__device__ __forceinline__ void sort8_desc(uint32_t (&k)[8])
+{
+#define ECCO_CMPX(a, b)                    \
+    {                                      \
+        const uint32_t hi = max(k[a], k[b]); \
+        k[b] = min(k[a], k[b]);            \
+        k[a] = hi;                         \
+    }
+    ECCO_CMPX(0, 1) ECCO_CMPX(2, 3) ECCO_CMPX(4, 5) ECCO_CMPX(6, 7)
+    ECCO_CMPX(0, 2) ECCO_CMPX(1, 3) ECCO_CMPX(4, 6) ECCO_CMPX(5, 7)
+    ECCO_CMPX(1, 2) ECCO_CMPX(5, 6)
+    ECCO_CMPX(0, 4) ECCO_CMPX(1, 5) ECCO_CMPX(2, 6) ECCO_CMPX(3, 7)
+    ECCO_CMPX(2, 4) ECCO_CMPX(3, 5)
+    ECCO_CMPX(1, 2) ECCO_CMPX(3, 4) ECCO_CMPX(5, 6)
+#undef ECCO_CMPX
+}
+
 __device__ __forceinline__ int quantise(const uint32_t* R, float t7, float v)
 {
     int idx = (t7 < v) ? 8 : 0;
@@ -87,9 +105,9 @@ __device__ __forceinline__ int quantise(const uint32_t* R, float t7, float v)
 // within the group.  cent: centroids [64][16] (SEL = 1 only).
 template <int SEL, int G>
 __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, const uint32_t* rows,
-                                             const float* cent, uint32_t* buf,
-                                             const float2 (&ends)[kNPat / (G / 8)], const uint16_t* src,
-                                             uint8_t* dst, int hl, uint32_t gmask, int npat, Counters& cnt)
+                                             const float* cent, uint32_t* buf, uint32_t* top,
+                                             const float2 (&ends)[4], const uint16_t* src, uint8_t* dst, int hl,
+                                             uint32_t gmask, int npat, Counters& cnt)
 {
     constexpr int kLanes = G / 8;             // lanes per group
     constexpr int kPatPerLane = kNPat / kLanes;
@@ -160,7 +178,9 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
 #pragma unroll
         for (int k = 0; k < kPatPerLane; ++k) {
             const int pat = hl + kLanes * k;
-            float d0 = __fsub_rn(umin, ends[k].x), d1 = __fsub_rn(umax, ends[k].y);
+            // 8 lanes (activation groups) hold 8 patterns each: read from L1 instead of registers
+            const float2 cp = (kPatPerLane <= 4) ? ends[k % 4] : __ldg(&tb->ends[pat]);
+            float d0 = __fsub_rn(umin, cp.x), d1 = __fsub_rn(umax, cp.y);
             float e = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
             const uint32_t ek = (pat < npat) ? __float_as_uint(e) : 0xffffffffu;
             if (ek < eb) {
@@ -251,27 +271,36 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     if (L <= kPayloadBits) {
         const int n = min(kMaxRec, (kPayloadBits - L) / kRecBits);
         if (n > 0) {
+            // candidates: key + 1 (0 = the scale element / taken), each lane's 8
+            // sorted descending once (Batcher odd-even merge network); every round
+            // takes the largest head of the group's lanes into the shared list
+            // `top` and its lane pops it.  Then lane r < n writes record r: the key
+            // holds the element's bf16 bits and index, so nothing else is needed.
             uint32_t k[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) k[j] = (owner && j == mj) ? 0u : keyof(b[j], i0 + j) + 1u;
-            int at = kHdrBits + L;
-            for (int r = 0; r < n; ++r, at += kRecBits) {
-                uint32_t mine = 0;
+            sort8_desc(k);
+            for (int r = 0; r < n; ++r) {
+                const uint32_t bestk = hw_max(gmask, k[0]);
+                if (k[0] == bestk) {  // exactly one lane: keys are unique
+                    top[r] = bestk - 1u;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) mine = max(mine, k[j]);
-                const uint32_t bestk = hw_max(gmask, mine);
-                if (mine == bestk) {  // exactly one lane: keys are unique
-                    float uv = u[0];
-                    int i = i0;
+                    for (int j = 0; j < 7; ++j) k[j] = k[j + 1];
+                    k[7] = 0u;
+                }
+            }
+            __syncwarp(gmask);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (k[j] == bestk) {
-                            uv = u[j];
-                            i = i0 + j;
-                            k[j] = 0u;
-                        }
-                    float v = fminf(fmaxf(rintf(__fmul_rn(uv, 127.0f)), -127.0f), 127.0f);
+            for (int pass = 0; pass < kMaxRec / kLanes; ++pass) {  // 16-lane groups: 1 pass, 8-lane: 2
+                const int r = hl + pass * kLanes;
+                if (r < n) {
+                    const uint32_t key = top[r];
+                    const int i = 127 - (int)((key >> 1) & 127u);
+                    const uint32_t xb = ((key >> 8) & 0x7fffu) | ((key & 1u) << 15);
+                    const float uv = __fmul_rn(bf16_bits_to_f32(xb), inv);
+                    const float v = fminf(fmaxf(rintf(__fmul_rn(uv, 127.0f)), -127.0f), 127.0f);
                     const uint32_t rec = (uint32_t)i | (((uint32_t)(int)v & 0xffu) << 7);
+                    const int at = kHdrBits + L + r * kRecBits;
                     const int ww = at >> 5, ss = at & 31;
                     atomicOr(&buf[ww], rec << ss);
                     if (ss > 32 - kRecBits) atomicOr(&buf[ww + 1], rec >> (32 - ss));
@@ -324,11 +353,13 @@ __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_
     __shared__ uint32_t rows[kNPat * kRow];
     __shared__ float cent[SEL ? kNPat * 16 : 1];  // C[p][j] pattern-major (full-MSE selection)
     __shared__ uint32_t bufs[kGpw * kEncWarps][20];
+    __shared__ uint32_t tops[kGpw * kEncWarps][kMaxRec];  // a group's outlier keys, in record order
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < kGpw * kEncWarps * 20; i += blockDim.x) (&bufs[0][0])[i] = 0u;
     const int sub = lane / kLanes, hl = lane % kLanes;
     const uint32_t gmask = (uint32_t)((1ull << kLanes) - 1ull) << (kLanes * sub);
     uint32_t* buf = bufs[kGpw * warp + sub];
+    uint32_t* top = tops[kGpw * warp + sub];
     Counters cnt = {0, 0, 0, 0, 0, 0, 0ull};
 
     const int64_t share = (P.total + gridDim.x - 1) / gridDim.x;
@@ -367,9 +398,9 @@ __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_
         if constexpr (SEL == 1) {
             for (int i = tid; i < kNPat * 16; i += blockDim.x) cent[i] = tb->Ct[i & 15][i >> 4];
         }
-        float2 ends[kNPat / kLanes];
+        float2 ends[4];  // this lane's patterns (16-lane groups); 8-lane groups read them on the fly
 #pragma unroll
-        for (int k = 0; k < kNPat / kLanes; ++k) ends[k] = __ldg(&tb->ends[hl + kLanes * k]);
+        for (int k = 0; k < 4; ++k) ends[k] = (kNPat / kLanes <= 4) ? __ldg(&tb->ends[hl + kLanes * k]) : float2{};
         __syncthreads();
 
         constexpr int kPerRound = kGpw * kEncWarps;  // groups per CTA round
@@ -381,7 +412,7 @@ __global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_
         for (; item < end; item += kPerRound) {
             const uint16_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * G;
             uint8_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * ECCO_BLOCK_BYTES;
-            encode_group<SEL, G>(tb, rows, cent, buf, ends, src, dst, hl, gmask, P.npat, cnt);
+            encode_group<SEL, G>(tb, rows, cent, buf, top, ends, src, dst, hl, gmask, P.npat, cnt);
             g += stride_g;
             r += stride_r;
             if (g >= gpr) {
