@@ -11,7 +11,11 @@
 // turn out to be wrong.
 //
 // G = 64 is the activation format (64 values per 512-bit block, the review
-// page's 2x ratio for activations); everything else is shared.
+// page's 2x ratio for activations); everything else is shared.  Activation
+// blocks nearly always carry all 16 outlier records, so there the rows are
+// assembled in shared memory (one 144-byte row per thread, 768 threads), the
+// records patch the row there, and the row goes out with full 32-byte stores
+// instead of 16 scattered 2-byte ones.
 //
 // Per block: parse the header (scale code, pattern, codebook), form the 16
 // output values bf16(s * C[p][j]) as register byte planes, decode the stream
@@ -22,13 +26,23 @@
 namespace ecco {
 namespace {
 
-constexpr int kDecThreads = 1024;
-constexpr int kWordStride = kDecThreads;  // word k of thread t at k * stride + t: conflict-free
-
 constexpr size_t kDecSmemLut = sizeof(((DevTables*)0)->lut);  // 65536
 constexpr size_t kDecSmemCt = sizeof(((DevTables*)0)->Ct);    // 4096
-constexpr size_t kDecSmemWords = 16 * kWordStride * 4;
-constexpr size_t kDecSmem = kDecSmemLut + kDecSmemCt + kDecSmemWords;
+constexpr int kRowWords = 36;  // staged 64-value row: 32 words + 4 pad (16-byte stores conflict-free)
+
+// Threads per CTA; word k of thread t's block at k * threads + t (conflict-free).
+template <int G>
+constexpr int dec_threads()
+{
+    return G == kG ? 1024 : 768;
+}
+
+template <int G>
+constexpr size_t dec_smem()
+{
+    return kDecSmemLut + kDecSmemCt + (size_t)16 * dec_threads<G>() * 4 +
+           (G == kG ? 0 : (size_t)dec_threads<G>() * kRowWords * 4);
+}
 
 // WIDE: 32-byte stores (output 32-byte aligned), else 16-byte stores.
 template <bool WIDE>
@@ -65,14 +79,17 @@ struct DecParams {
 // segment by segment, restaging the segment's tables in shared memory when
 // its share crosses into the next segment.
 template <bool WIDE, int MAXSEG, int G>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecParams<MAXSEG> P)
+__global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __grid_constant__ DecParams<MAXSEG> P)
 {
+    constexpr int kDecThreads = dec_threads<G>(), kWordStride = kDecThreads;
+    constexpr bool kRows = G != kG;  // rows assembled in shared memory
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kDecSmemLut);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kDecSmemLut + kDecSmemCt);
     const int tid = threadIdx.x;
     uint32_t* ws = s_w + tid;
+    uint32_t* row = s_w + 16 * kWordStride + tid * kRowWords;  // kRows only
 
     const int64_t share = (P.total + gridDim.x - 1) / gridDim.x;
     int64_t lo = (int64_t)blockIdx.x * share;
@@ -134,7 +151,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 uint32_t wa[4], wb[4];
                 chunk_values(st, lut, ws, kWordStride, vp, wa);
                 chunk_values(st, lut, ws, kWordStride, vp, wb);
-                store16<WIDE>(dst + 16 * c, wa, wb);
+                if constexpr (kRows) {
+                    *reinterpret_cast<uint4*>(row + 8 * c) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                    *reinterpret_cast<uint4*>(row + 8 * c + 4) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                } else {
+                    store16<WIDE>(dst + 16 * c, wa, wb);
+                }
             }
 
             if (st.room >= 0) {  // unclipped: outlier records follow the codewords
@@ -145,7 +167,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                     int i = (int)(rec & (uint32_t)(G - 1));  // the 7-bit index, modulo G
                     int qv = (int)(int8_t)(uint8_t)(rec >> 7);
                     float o = __fdiv_rn((float)qv, 127.0f);
-                    dst[i] = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
+                    const uint16_t v = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
+                    if constexpr (kRows)
+                        reinterpret_cast<uint16_t*>(row)[i] = v;
+                    else
+                        dst[i] = v;
+                }
+            }
+            if constexpr (kRows) {
+#pragma unroll
+                for (int c = 0; c < G / 16; ++c) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(row + 8 * c);
+                    const uint4 b = *reinterpret_cast<const uint4*>(row + 8 * c + 4);
+                    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+                    store16<WIDE>(dst + 16 * c, wa, wb);
                 }
             }
         }
@@ -161,14 +196,14 @@ cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
     cudaGetDevice(&dev);
     if (configured != dev) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<WIDE, MAXSEG, G>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmem);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dec_smem<G>());
         if (e != cudaSuccess) return e;
         configured = dev;
     }
-    int64_t want = (P.total + kDecThreads - 1) / kDecThreads;
+    int64_t want = (P.total + dec_threads<G>() - 1) / dec_threads<G>();
     int64_t cap = device_sm_count();
     int grid = (int)(want < cap ? want : cap);
-    decode_kernel<WIDE, MAXSEG, G><<<grid, kDecThreads, kDecSmem, s>>>(P);
+    decode_kernel<WIDE, MAXSEG, G><<<grid, dec_threads<G>(), dec_smem<G>(), s>>>(P);
     return cudaGetLastError();
 }
 

@@ -154,3 +154,18 @@ def test_attention_argument_errors():
     assert call(n=0) == _lib.ECCO_ERR_ARG
     assert call(ws_bytes=4 * 130 * 4 - 1) == _lib.ECCO_ERR_ARG
     assert call(kptr=kb.data_ptr() + 8) == _lib.ECCO_ERR_ALIGN
+
+
+def test_attention_on_garbage_blocks():
+    """Random K and V blocks (clipped streams, duplicate record indexes, null
+    scale codes) against the oracle's attention over its own decoding."""
+    B, H, G, S_cap, n = 1, 2, 4, 777, 700
+    kt, vt = table_set("learned_kv"), table_set("random1")
+    rng = np.random.default_rng(9)
+    kb = rng.integers(0, 256, (B, H, S_cap, 64), dtype=np.uint8)
+    vb = rng.integers(0, 256, (B, H, S_cap, 64), dtype=np.uint8)
+    q = q_bits(B, H * G, seed=10)
+    scale = 1e-3  # random scales make huge scores; keep the softmax finite
+    ref, aw = oracle.attention(kt, vt, kb, vb, q, n, scale)
+    assert np.isfinite(ref).all()
+    check(run(kt, vt, kb, vb, q, n, scale), ref, aw)
