@@ -347,7 +347,7 @@ struct EncParams {  // by value: no device-side segment table
 // Each CTA encodes one contiguous, equal share of all groups of the launch,
 // segment by segment, restaging the pattern rows when it enters a new segment.
 template <int MAXSEG, int SEL, int G>
-__global__ void __launch_bounds__(kEncWarps * 32, 3) encode_kernel(const __grid_constant__ EncParams<MAXSEG> P)
+__global__ void __launch_bounds__(kEncWarps * 32, 4) encode_kernel(const __grid_constant__ EncParams<MAXSEG> P)
 {
     constexpr int kLanes = G / 8, kGpw = 32 / kLanes;  // lanes per group, groups per warp
     __shared__ uint32_t rows[kNPat * kRow];
@@ -439,7 +439,7 @@ cudaError_t run_encode(const EncParams<MAXSEG>& P, int select, cudaStream_t s)
 {
     const int per_cta = (32 / (G / 8)) * kEncWarps;
     int64_t want = (P.total + per_cta - 1) / per_cta;
-    int64_t cap = (int64_t)device_sm_count() * 3;  // resident CTAs at 3 per SM
+    int64_t cap = (int64_t)device_sm_count() * 4;  // resident CTAs at 4 per SM
     int grid = (int)(want < cap ? want : cap);
     if (select == ECCO_SELECT_MSE)
         encode_kernel<MAXSEG, 1, G><<<grid, kEncWarps * 32, 0, s>>>(P);
