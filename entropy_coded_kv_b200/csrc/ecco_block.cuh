@@ -98,6 +98,7 @@ __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, cons
     uint32_t nib = 0;
     int used = 0;
     kv = 0;
+    const uint32_t lut_sh = (uint32_t)__cvta_generic_to_shared(lut);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         refill(st, ws, stride);
@@ -105,7 +106,8 @@ __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, cons
         int u = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            uint32_t e = lut[cur & 0xffu];
+            uint32_t e;  // the table is written before a CTA barrier: no ordering needed here
+            asm("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(lut_sh + (cur & 0xffu)));
             uint32_t len = e >> 4;
             nib = __funnelshift_r(nib, e, 4);  // symbol into the top nibble; the first ends at the bottom
             cur >>= len;
