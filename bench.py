@@ -821,7 +821,7 @@ def time_oracle(sample, nthreads):
     if "attn" in sample:
         (kt, vt), (kb, vb), qb, S, scale = sample["attn"]
         n = kb.shape[0]
-        oracle.attention(kt, vt, kb.reshape(n, 1, S, 64), vb.reshape(n, 1, S, 64), qb, S, scale)
+        oracle.attention(kt, vt, kb.reshape(n, 1, S, 64), vb.reshape(n, 1, S, 64), qb, S, scale, nthreads=nthreads)
     return time.perf_counter() - t0
 
 
@@ -836,8 +836,10 @@ def cpu_baseline(wl, target_s):
     while total < target_s and reps < 1000:
         total += time_oracle(sample, cores)
         reps += 1
+    one = time_oracle(sample, 1)  # the same sample on one host thread, once
     return {"value": sample["bytes"] * reps / total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{sample['what']}, {reps} repetitions", "seconds": round(total, 2)}
+            "sample": f"{sample['what']}, {reps} repetitions", "seconds": round(total, 2),
+            "value_1_thread": round(sample["bytes"] / one / 1e9, 4)}
 
 
 # ------------------------------------------------------------------ main

@@ -262,14 +262,15 @@ def gemv(tables, blocks, rows: int, cols: int, x):
     return y, ya
 
 
-def attention(k_tables, v_tables, k_blocks, v_blocks, q, seq_len: int, scale: float):
+def attention(k_tables, v_tables, k_blocks, v_blocks, q, seq_len: int, scale: float, nthreads: int = 1):
     """Decode-phase attention over a compressed KV cache, in fp64.
 
     k_blocks / v_blocks: [B, Hkv, S_cap, 64] uint8 (token s of head h at [b, h, s]);
     q: bf16 bits [B, Hkv * G, 128] (query head j uses KV head j // G).
     K~, V~ are this oracle's decoded bf16 values; then, per query head,
     softmax over the first seq_len tokens of (q . k~) * scale, and out = sum p v~.
-    Returns (out [B, Hq, 128] fp64, abs_weighted [B, Hq, 128] = sum_s p_s |v~_s|)."""
+    Returns (out [B, Hq, 128] fp64, abs_weighted [B, Hq, 128] = sum_s p_s |v~_s|).
+    nthreads: threads for the block decoding (the attention itself is numpy)."""
     kb = np.ascontiguousarray(np.asarray(k_blocks, dtype=np.uint8))
     vb = np.ascontiguousarray(np.asarray(v_blocks, dtype=np.uint8))
     B, H, _, _ = kb.shape
@@ -280,8 +281,8 @@ def attention(k_tables, v_tables, k_blocks, v_blocks, q, seq_len: int, scale: fl
     aw = np.zeros((B, Hq, G))
     for b in range(B):
         for h in range(H):
-            K = decode(k_tables, kb[b, h, :seq_len]).astype(np.uint32) << 16
-            V = decode(v_tables, vb[b, h, :seq_len]).astype(np.uint32) << 16
+            K = decode(k_tables, kb[b, h, :seq_len], nthreads).astype(np.uint32) << 16
+            V = decode(v_tables, vb[b, h, :seq_len], nthreads).astype(np.uint32) << 16
             Kf = K.view(np.float32).astype(np.float64)
             Vf = V.view(np.float32).astype(np.float64)
             for j in range(h * grp, (h + 1) * grp):
