@@ -64,7 +64,7 @@ constexpr size_t kOffQf = kOffX + (size_t)kAtWarps * 32 * kHeads * 4;         //
 constexpr size_t kOffQb = kOffQf + (size_t)kHeads * 128 * 4;                  // [head][kQbRow] bf16
 constexpr size_t kOffRed = kOffQb + (size_t)kHeads * kQbRow * 2;              // [2][warp][head] f32
 constexpr size_t kOffAcc = kOffRed + (size_t)2 * kAtWarps * kHeads * 4;       // [head][128] f32
-constexpr size_t kAttnSmem = kOffAcc + (size_t)kHeads * 128 * 4;
+constexpr size_t kAttnSmem = kOffAcc + (size_t)kHeads * 128 * 4 + kSmemAlign;
 static_assert(kOffQb % 16 == 0 && kOffRed % 16 == 0 && kOffAcc % 16 == 0, "alignment");
 
 __device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -162,7 +162,8 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)
 template <int G>
 __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_constant__ AttnArgs A)
 {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t* smem = aligned_smem(smem_raw);
     uint8_t* s_lut = smem + kOffLut;
     float* s_Ct = reinterpret_cast<float*>(smem + kOffCt);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kOffWords);

@@ -91,6 +91,8 @@ __device__ __forceinline__ void refill(Stream& st, const uint32_t* ws, int strid
 // Decodes 8 symbols.  Returns their nibbles (symbol k in bits 4k..4k+3); `kv`
 // = number of them that end
 // at or before bit 512 (8 unless CHECK and the block clips here or earlier).
+// `lut` must start on a 256-byte boundary of the shared window (aligned_smem):
+// the lookup address is the table base OR-ed with the next 8 stream bits.
 template <bool CHECK>
 __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, const uint32_t* ws, int stride,
                                             int& kv)
@@ -107,7 +109,7 @@ __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, cons
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             uint32_t e;  // the table is written before a CTA barrier: no ordering needed here
-            asm("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(lut_sh + (cur & 0xffu)));
+            asm("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(lut_sh | (cur & 0xffu)));
             uint32_t len = e >> 4;
             nib = __funnelshift_r(nib, e, 4);  // symbol into the top nibble; the first ends at the bottom
             cur >>= len;
@@ -133,16 +135,18 @@ __device__ __forceinline__ void mask_tail(uint32_t w[4], int kv)
     }
 }
 
-// Decodes one chunk into 4 bf16x2 words; also returns the nibbles.
+// Decodes one chunk into 4 bf16x2 words; also returns the nibbles.  The
+// lanes that run together take the checked walk as soon as one of them is
+// within 64 bits of the end (a vote), so a warp never runs both walks.
 __device__ __forceinline__ uint32_t chunk_values(Stream& st, const uint8_t* lut, const uint32_t* ws, int stride,
                                                  const ValuePlanes& vp, uint32_t w[4])
 {
     int kv;
     uint32_t nib;
-    if (st.room >= 64)
-        nib = decode8<false>(st, lut, ws, stride, kv);
-    else
+    if (__any_sync(__activemask(), st.room < 64))
         nib = decode8<true>(st, lut, ws, stride, kv);
+    else
+        nib = decode8<false>(st, lut, ws, stride, kv);
     uint32_t sh4 = nib << 4;
     planes_to_bf16<0>(vp, nib, sh4, w[0], w[1]);
     planes_to_bf16<1>(vp, nib, sh4, w[2], w[3]);
@@ -176,6 +180,17 @@ __device__ __forceinline__ void stage_words(uint32_t* ws, int stride, const uint
     ws[13 * stride] = q3.y;
     ws[14 * stride] = q3.z;
     ws[15 * stride] = q3.w;
+}
+
+// Kernels that walk blocks reserve kSmemAlign bytes more than their layout
+// needs and lay it out from aligned_smem(): the decode tables then start on a
+// 256-byte boundary of the shared window, as decode8 requires.
+constexpr size_t kSmemAlign = 256;
+
+__device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw)
+{
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(raw);
+    return raw + ((uint32_t)kSmemAlign - (a & ((uint32_t)kSmemAlign - 1u))) % (uint32_t)kSmemAlign;
 }
 
 // Copies a tensor's decode tables (65,536 B) and transposed centroids (4,096 B)

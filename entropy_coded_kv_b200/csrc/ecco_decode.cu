@@ -40,7 +40,7 @@ constexpr int dec_threads()
 template <int G>
 constexpr size_t dec_smem()
 {
-    return kDecSmemLut + kDecSmemCt + (size_t)16 * dec_threads<G>() * 4 +
+    return kSmemAlign + kDecSmemLut + kDecSmemCt + (size_t)16 * dec_threads<G>() * 4 +
            (G == kG ? 0 : (size_t)dec_threads<G>() * kRowWords * 4);
 }
 
@@ -83,7 +83,8 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
 {
     constexpr int kDecThreads = dec_threads<G>(), kWordStride = kDecThreads;
     constexpr bool kRows = G != kG;  // rows assembled in shared memory
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t* smem = aligned_smem(smem_raw);
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kDecSmemLut);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kDecSmemLut + kDecSmemCt);
@@ -160,13 +161,17 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
             }
 
             if (st.room >= 0) {  // unclipped: outlier records follow the codewords
+                // The walk ended exactly at the first record, so the stream
+                // window reads them in order.  q / 127 is divided here (an
+                // ALU sequence) rather than looked up: the kernel is bound by
+                // the L1 data path, which a table gather would load further.
                 const int n = min(kMaxRec, st.room / kRecBits);
-                int at = kBlockBits - st.room;
-                for (int k = 0; k < n; ++k, at += kRecBits) {
-                    uint32_t rec = read_record(ws, kWordStride, at);
-                    int i = (int)(rec & (uint32_t)(G - 1));  // the 7-bit index, modulo G
-                    int qv = (int)(int8_t)(uint8_t)(rec >> 7);
-                    float o = __fdiv_rn((float)qv, 127.0f);
+                for (int k = 0; k < n; ++k) {
+                    refill(st, ws, kWordStride);
+                    const uint32_t rec = __funnelshift_r(st.lo, st.hi, st.b);
+                    st.b += kRecBits;
+                    const int i = (int)(rec & (uint32_t)(G - 1));  // the 7-bit index, modulo G
+                    const float o = __fdiv_rn((float)(int)(int8_t)(uint8_t)(rec >> 7), 127.0f);
                     const uint16_t v = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
                     if constexpr (kRows)
                         reinterpret_cast<uint16_t*>(row)[i] = v;

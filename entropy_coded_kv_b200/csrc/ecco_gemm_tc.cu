@@ -49,7 +49,7 @@ constexpr size_t kOffNib = kOffWords + 16 * kTcStride * 4;
 constexpr size_t kOffA = kOffNib + 16 * kTcThreads * 4;
 constexpr size_t kOffB = kOffA + (size_t)kTcTiles * 2 * kSliceBytes;
 constexpr size_t kOffBar = kOffB + (size_t)kMaxGroups * 8 * kBSliceBytes;
-constexpr size_t kTcSmem = kOffBar + 128;
+constexpr size_t kTcSmem = kOffBar + 128 + kSmemAlign;
 
 // Instruction descriptor: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12
 // = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -129,7 +129,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    int64_t gpr, const uint16_t* __restrict__ x, int batch, int64_t cols, int splits,
                    float* __restrict__ y)
 {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    uint8_t* smem = aligned_smem(smem_raw);
     uint8_t* s_lut = smem + kOffLut;
     float* s_Ct = reinterpret_cast<float*>(smem + kOffCt);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kOffWords);
@@ -231,13 +232,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (s != 0.0f && st.room >= 0) {  // outlier records: add (new - old) * x
             const int n = min(kMaxRec, st.room / kRecBits);
             const int at0 = kBlockBits - st.room;
-            for (int k = n - 1; k >= 0; --k) {  // the last record of an element wins
+            // Newest first: the last record of an element wins, so an element
+            // already seen (128-bit mask) is skipped.
+            uint32_t seen0 = 0u, seen1 = 0u, seen2 = 0u, seen3 = 0u;
+            for (int k = n - 1; k >= 0; --k) {
                 uint32_t rec = read_record(ws, kTcStride, at0 + k * kRecBits);
                 int i = (int)(rec & 127u);
-                bool later = false;
-                for (int k2 = k + 1; k2 < n; ++k2)
-                    later = later || ((int)(read_record(ws, kTcStride, at0 + k2 * kRecBits) & 127u) == i);
-                if (later) continue;
+                const uint32_t bit = 1u << (i & 31), q = (uint32_t)i >> 5;
+                const uint32_t was = (q == 0u ? seen0 : q == 1u ? seen1 : q == 2u ? seen2 : seen3) & bit;
+                seen0 |= (q == 0u) ? bit : 0u;
+                seen1 |= (q == 1u) ? bit : 0u;
+                seen2 |= (q == 2u) ? bit : 0u;
+                seen3 |= (q == 3u) ? bit : 0u;
+                if (was) continue;
                 float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __ldg(&tb->o_of_q[rec >> 7]))));
                 uint32_t osym = (nibs[(i >> 3) * kTcThreads] >> (4 * (i & 7))) & 15u;
                 uint32_t ow = (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);

@@ -37,7 +37,7 @@ constexpr int gv_threads()
 template <int B>
 constexpr size_t gv_smem()
 {
-    return kGvLut + kGvCt + (size_t)16 * gv_threads<B>() * 4 * 2 + (size_t)kGvWin * kG * B * 4;
+    return kSmemAlign + kGvLut + kGvCt + (size_t)16 * gv_threads<B>() * 4 * 2 + (size_t)kGvWin * kG * B * 4;
 }
 
 template <int B>
@@ -47,7 +47,8 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
                 float* __restrict__ y)
 {
     constexpr int kGvThreads = gv_threads<B>(), kGvStride = kGvThreads;
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t* smem = aligned_smem(smem_raw);
     uint8_t* s_lut = smem;
     float* s_Ct = reinterpret_cast<float*>(smem + kGvLut);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kGvLut + kGvCt);
@@ -118,7 +119,16 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
         for (int c = 0; c < 16; ++c) {
             uint32_t w[4];
             nibs[c * kGvThreads] = chunk_values(st, lut, ws, kGvStride, vp, w);
-            const float* xk = xs + c * 8 * B;
+            // the chunk's 8 x B inputs as 16-byte broadcast loads (one L1 wavefront each)
+            float xk[8 * B];
+#pragma unroll
+            for (int v4 = 0; v4 < 2 * B; ++v4) {
+                const float4 t = reinterpret_cast<const float4*>(xs + c * 8 * B)[v4];
+                xk[4 * v4] = t.x;
+                xk[4 * v4 + 1] = t.y;
+                xk[4 * v4 + 2] = t.z;
+                xk[4 * v4 + 3] = t.w;
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 float v = __uint_as_float((j & 1) ? (w[j >> 1] & 0xffff0000u) : (w[j >> 1] << 16));
@@ -129,14 +139,21 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
         if (s != 0.0f && st.room >= 0) {  // outlier records replace their element's value
             const int n = min(kMaxRec, st.room / kRecBits);
             const int at0 = kBlockBits - st.room;
-            for (int k = n - 1; k >= 0; --k) {  // the last record of an element wins
+            // Newest first: the last record of an element wins, so an element
+            // already seen (128-bit mask) is skipped.
+            uint32_t seen0 = 0u, seen1 = 0u, seen2 = 0u, seen3 = 0u;
+            for (int k = n - 1; k >= 0; --k) {
                 uint32_t rec = read_record(ws, kGvStride, at0 + k * kRecBits);
                 int i = (int)(rec & 127u);
-                bool later = false;
-                for (int k2 = k + 1; k2 < n; ++k2)
-                    later = later || ((int)(read_record(ws, kGvStride, at0 + k2 * kRecBits) & 127u) == i);
-                if (later) continue;
-                float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __ldg(&tb->o_of_q[rec >> 7]))));
+                const uint32_t bit = 1u << (i & 31), q = (uint32_t)i >> 5;
+                const uint32_t was = (q == 0u ? seen0 : q == 1u ? seen1 : q == 2u ? seen2 : seen3) & bit;
+                seen0 |= (q == 0u) ? bit : 0u;
+                seen1 |= (q == 1u) ? bit : 0u;
+                seen2 |= (q == 2u) ? bit : 0u;
+                seen3 |= (q == 3u) ? bit : 0u;
+                if (was) continue;
+                float nv = bf16_bits_to_f32(
+                    f32_to_bf16_bits(__fmul_rn(s, __fdiv_rn((float)(int)(int8_t)(uint8_t)(rec >> 7), 127.0f))));
                 uint32_t osym = (nibs[(i >> 3) * kGvThreads] >> (4 * (i & 7))) & 15u;
                 uint32_t ow = (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);
                 uint32_t oh = (osym < 8) ? ((osym < 4) ? vp.hi[0] : vp.hi[1]) : ((osym < 12) ? vp.hi[2] : vp.hi[3]);
