@@ -10,7 +10,7 @@ workloads: `c1` (256 x 1024 matrix, encode + decode), `mlp` (14336 x 4096
 weight: encode, decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights,
 encode and decode of the whole set), `longctx` (32 layers x K,V x
 [1, 8, 131072, 128]: full streaming decode plus a one-token append per layer),
-`attn` (one-token append + fused decode+attention over the compressed cache of
+`attn` (one-token append + staged decode+attention over the compressed cache of
 the `kv` layer, 32 query heads), `select` (encode of the `kv` layer with
 full-MSE pattern selection, plus a quality study of min/max vs full-MSE
 selection with 64 and 16 patterns), `act` (the 2x activation format: [8192,
@@ -546,7 +546,8 @@ class AttnWorkload(Workload):
         self.torch, self.ecco, self.dev = torch, ecco, dev
         self.desc = ("decode-phase attention over a compressed Llama-3-8B-shaped layer KV cache: K, V "
                      "[8, 8, 4096, 128] as 64-byte blocks, 32 query heads (group 4); a step appends one "
-                     "token's K and V (128 groups) and runs fused decode+attention over all 4096 tokens")
+                     "token's K and V (128 groups) and runs staged decode+attention over all 4096 tokens "
+                     "(block decoder into a workspace scratch, then the split kernel)")
         K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
         Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
         self.tables = [ecco.Tables(learn_tables(Kc, seed=0), dev), ecco.Tables(learn_tables(Vc, seed=0), dev)]
@@ -561,14 +562,15 @@ class AttnWorkload(Workload):
         g = torch.Generator(device=dev).manual_seed(77 + seed_offset)
         self.q = torch.randn(self.B, self.H * self.G, self.D, generator=g, device=dev).to(torch.bfloat16)
         self.out = torch.empty(self.B, self.H * self.G, self.D, dtype=torch.float32, device=dev)
-        self.ws = torch.empty(ecco.attention_workspace_bytes(self.B, self.H, self.G, self.S), dtype=torch.uint8,
-                              device=dev)
+        self.ws = torch.empty(ecco.attention_staged_workspace_bytes(self.B, self.H, self.G, self.S),
+                              dtype=torch.uint8, device=dev)
         self.scale = 1.0 / self.D ** 0.5
-        self.launches_per_step = 3  # append (one multi-segment launch), split kernel, merge kernel
-        self.api = "entropy_coded_kv_b200.encode_multi/decode_attention (C ABI) with pinned host buffers"
+        # append (one multi-segment launch); one chunk: decode (K and V in one launch), split kernel; merge
+        self.launches_per_step = 4
+        self.api = "entropy_coded_kv_b200.encode_multi/decode_attention_staged (C ABI) with pinned host buffers"
         self.att_ms = []
 
-    def bytes_decoded(self):  # bf16 K and V bytes the attention kernel decodes (consumed on chip)
+    def bytes_decoded(self):  # bf16 K and V bytes the step decodes
         return 2 * self.n * 256
 
     def bytes_encoded(self):
@@ -578,8 +580,8 @@ class AttnWorkload(Workload):
         return 1.0 / 64
 
     def _attend(self, q):
-        return self.ecco.decode_attention(self.blocks[0], self.blocks[1], self.tables[0], self.tables[1], q,
-                                          self.S, self.scale, out=self.out, workspace=self.ws)
+        return self.ecco.decode_attention_staged(self.blocks[0], self.blocks[1], self.tables[0], self.tables[1], q,
+                                                 self.S, self.scale, out=self.out, workspace=self.ws)
 
     def step(self, record=False):
         self.ecco.encode_multi(self.app)
@@ -596,7 +598,7 @@ class AttnWorkload(Workload):
         self.torch.cuda.synchronize()
         ms = [a.elapsed_time(b) for a, b in self.att_ms]
         nbytes = 2 * self.n * 64 + self.q.numel() * 2 + self.out.numel() * 4
-        return "attn_split_kernel+attn_merge_kernel", nbytes, ms
+        return "decode_kernel+attn_split_kernel+attn_merge_kernel", nbytes, ms
 
     def e2e_setup(self):
         torch = self.torch
@@ -973,7 +975,7 @@ KERNEL_SOURCES = {
     "decode_kernel": ["ecco_decode.cu", "ecco_block.cuh"],
     "decode_kernel<G=64>": ["ecco_decode.cu", "ecco_block.cuh"],
     "encode_kernel<.,SEL=1>": ["ecco_encode.cu"],
-    "attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_block.cuh"],
+    "decode_kernel+attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_decode.cu", "ecco_block.cuh"],
 }
 
 

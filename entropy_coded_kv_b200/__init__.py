@@ -25,6 +25,7 @@ BLOCK_BYTES = 64
 
 __all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
            "decode_attention", "attention_workspace_bytes", "decode_attention_static",
+           "decode_attention_staged", "attention_staged_workspace_bytes",
            "encode_act", "decode_act", "GROUP_ACT", "learn_tables", "huffman_lengths",
            "new_stats", "read_stats", "flat_desc", "kv_append_desc", "EccoError", "Desc"]
 
@@ -169,6 +170,10 @@ def attention_workspace_bytes(batch: int, kv_heads: int, group: int, seq_len: in
     return int(_lib.load().ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len))
 
 
+def attention_staged_workspace_bytes(batch: int, kv_heads: int, group: int, seq_len: int) -> int:
+    return int(_lib.load().ecco_decode_attention_staged_workspace_bytes(batch, kv_heads, group, seq_len))
+
+
 def decode_attention(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: Tables, v_tables: Tables,
                      q: torch.Tensor, seq_len: int, scale: float, out: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None) -> torch.Tensor:
@@ -177,6 +182,21 @@ def decode_attention(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: T
     k_blocks / v_blocks: uint8 [B, Hkv, S_cap, 64]; q: bf16 [B, Hkv * G, 128].
     Returns fp32 [B, Hkv * G, 128]: softmax over the first seq_len tokens of
     scale * q . K~, applied to V~ (K~, V~ decoded inside the kernel)."""
+    return _attention("ecco_decode_attention", attention_workspace_bytes, k_blocks, v_blocks, k_tables,
+                      v_tables, q, seq_len, scale, out, workspace)
+
+
+def decode_attention_staged(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: Tables, v_tables: Tables,
+                            q: torch.Tensor, seq_len: int, scale: float, out: torch.Tensor | None = None,
+                            workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """decode_attention computed in stages: each chunk of tokens is decoded by
+    the block decoder into a scratch in the workspace (sized to stay in L2),
+    then attended.  Same arguments and result."""
+    return _attention("ecco_decode_attention_staged", attention_staged_workspace_bytes, k_blocks, v_blocks,
+                      k_tables, v_tables, q, seq_len, scale, out, workspace)
+
+
+def _attention(fn, ws_bytes, k_blocks, v_blocks, k_tables, v_tables, q, seq_len, scale, out, workspace):
     _check_tensor(k_blocks, torch.uint8, "k_blocks", k_tables.device)
     _check_tensor(v_blocks, torch.uint8, "v_blocks", v_tables.device)
     _check_tensor(q, torch.bfloat16, "q", k_tables.device)
@@ -189,16 +209,16 @@ def decode_attention(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_tables: T
     if out is None:
         out = torch.empty((B, H * G, GROUP), dtype=torch.float32, device=q.device)
     _check_tensor(out, torch.float32, "out", k_tables.device)
-    need = attention_workspace_bytes(B, H, G, seq_len)
+    need = ws_bytes(B, H, G, seq_len)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     _check_tensor(workspace, torch.uint8, "workspace", k_tables.device)
-    rc = _lib.load().ecco_decode_attention(
+    rc = getattr(_lib.load(), fn)(
         k_tables.handle, v_tables.handle, ctypes.c_void_p(k_blocks.data_ptr()),
         ctypes.c_void_p(v_blocks.data_ptr()), s_cap, B, H, G, int(seq_len), ctypes.c_void_p(q.data_ptr()),
         float(scale), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel(), _stream(q.device))
-    _lib.check(rc, "ecco_decode_attention")
+    _lib.check(rc, fn)
     return out
 
 

@@ -28,6 +28,7 @@ EXPORTED = [
     "ecco_abi_version", "ecco_device_timeouts", "ecco_decode_attention",
     "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static", "ecco_select_encode_ex",
     "ecco_select_encode_act", "ecco_decode_act", "ecco_learn_tables", "ecco_huffman_lengths",
+    "ecco_decode_attention_staged", "ecco_decode_attention_staged_workspace_bytes",
 ]
 
 
@@ -82,10 +83,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_decode_attention_static.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P]
     L.ecco_decode_attention.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P,
                                         ctypes.c_size_t, P]
+    L.ecco_decode_attention_staged_workspace_bytes.argtypes = [I, I, I, I]
+    L.ecco_decode_attention_staged.argtypes = L.ecco_decode_attention.argtypes
+    sizes = ("ecco_decode_attention_workspace_bytes", "ecco_decode_attention_staged_workspace_bytes")
     for fn in EXPORTED:
-        if fn not in ("ecco_strerror", "ecco_decode_attention_workspace_bytes"):
+        if fn != "ecco_strerror" and fn not in sizes:
             getattr(L, fn).restype = I
-    L.ecco_decode_attention_workspace_bytes.restype = ctypes.c_size_t
+    for fn in sizes:
+        getattr(L, fn).restype = ctypes.c_size_t
     _lib = L
     return L
 

@@ -197,6 +197,48 @@ extern "C" int ecco_decode_attention(const ecco_tables* kt, const ecco_tables* v
                                    out, static_cast<float*>(ws), (cudaStream_t)stream));
 }
 
+namespace {
+constexpr size_t kScratchAlign = 256;
+size_t staged_partials_bytes(int batch, int kv_heads, int group, int seq_len)
+{
+    const size_t p = ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len);
+    return (p + kScratchAlign - 1) / kScratchAlign * kScratchAlign;
+}
+}  // namespace
+
+extern "C" size_t ecco_decode_attention_staged_workspace_bytes(int batch, int kv_heads, int group, int seq_len)
+{
+    if (ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len) == 0) return 0;
+    const size_t chunk = (size_t)ecco::staged_chunk_tokens(batch, kv_heads, seq_len);
+    return staged_partials_bytes(batch, kv_heads, group, seq_len) + kScratchAlign +
+           2 * (size_t)batch * (size_t)kv_heads * chunk * 128 * sizeof(uint16_t);
+}
+
+extern "C" int ecco_decode_attention_staged(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                                            const uint8_t* vblk, int64_t s_cap, int batch, int kv_heads,
+                                            int group, int seq_len, const uint16_t* q, float scale, float* out,
+                                            void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_tables(kt);
+    if (rc) return rc;
+    if ((rc = check_tables(vt))) return rc;
+    if (batch < 1 || kv_heads < 1 || group < 1 || group > 8 || seq_len < 1 || s_cap < seq_len)
+        return ECCO_ERR_ARG;
+    if ((int64_t)batch * kv_heads > 65535 || s_cap > ((int64_t)1 << 34)) return ECCO_ERR_ARG;
+    if (!kblk || !vblk || !q || !out || !ws) return ECCO_ERR_ARG;
+    if (ws_bytes < ecco_decode_attention_staged_workspace_bytes(batch, kv_heads, group, seq_len))
+        return ECCO_ERR_ARG;
+    if (!aligned16(kblk) || !aligned16(vblk) || (reinterpret_cast<uintptr_t>(q) & 1u) ||
+        (reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 3u))
+        return ECCO_ERR_ALIGN;
+    // partials first, then the decoded-row scratch from the next 256-byte boundary
+    const uintptr_t sc = (reinterpret_cast<uintptr_t>(ws) + staged_partials_bytes(batch, kv_heads, group, seq_len) +
+                          kScratchAlign - 1) / kScratchAlign * kScratchAlign;
+    return status(launch_attention_staged(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, scale,
+                                          out, static_cast<float*>(ws), reinterpret_cast<uint16_t*>(sc),
+                                          (cudaStream_t)stream));
+}
+
 extern "C" int ecco_learn_tables(const uint16_t* x, int64_t n_groups, int group, int n_patterns, uint64_t seed,
                                  void* blob, size_t blob_bytes, void* stream)
 {

@@ -51,6 +51,13 @@ struct AttnArgs {
     const uint16_t* q;
     float scale;
     float* ws;  // [B][H*G][splits][130]: 128 partial p.V, then max, sum
+    // Staged path only: the current chunk's decoded K and V rows (bf16,
+    // [B*H][cstride][128]), its first token c0 (a multiple of 512) and the
+    // index of its first split.
+    const uint16_t* kx;
+    const uint16_t* vx;
+    int64_t c0, cstride;
+    int split0;
 };
 
 // shared memory map (bytes)
@@ -66,6 +73,25 @@ constexpr size_t kOffRed = kOffQb + (size_t)kHeads * kQbRow * 2;              //
 constexpr size_t kOffAcc = kOffRed + (size_t)2 * kAtWarps * kHeads * 4;       // [head][128] f32
 constexpr size_t kAttnSmem = kOffAcc + (size_t)kHeads * 128 * 4 + kSmemAlign;
 static_assert(kOffQb % 16 == 0 && kOffRed % 16 == 0 && kOffAcc % 16 == 0, "alignment");
+// Staged path: no tables, stream words or nibbles; each warp's tile holds its
+// 32 tokens' whole decoded rows (filled by cp.async), 272 B apart so that
+// ldmatrix rows fall on distinct banks.
+constexpr int kFullRow = 68;  // words per staged full row: 128 bf16 + 16 B pad
+constexpr size_t kSOffTile = 0;
+constexpr size_t kSOffQf = kSOffTile + (size_t)kAtWarps * 32 * kFullRow * 4;
+constexpr size_t kSOffQb = kSOffQf + (size_t)kHeads * 128 * 4;
+constexpr size_t kSOffRed = kSOffQb + (size_t)kHeads * kQbRow * 2;
+constexpr size_t kSOffAcc = kSOffRed + (size_t)2 * kAtWarps * kHeads * 4;
+constexpr size_t kAttnSmemStaged = kSOffAcc + (size_t)kHeads * 128 * 4 + kSmemAlign;
+static_assert(kSOffQb % 16 == 0 && kSOffRed % 16 == 0 && kSOffAcc % 16 == 0, "alignment");
+
+// Tokens per chunk of the staged path: the decoded K and V rows of a chunk
+// (2 x rows x chunk x 256 B) stay within kStagedScratchBytes; a multiple of
+// 512 (whole splits).  Measured on B200 ([8, 8, 4096] and [1, 8, 131072]
+// caches): chunks that fit in L2 (32 MiB) are slower than one large chunk,
+// because a decoder launch needs several blocks per thread to hide its serial
+// walk, so the bound is set by memory use, not by L2.
+constexpr int64_t kStagedScratchBytes = 1024ll << 20;
 
 __device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1)
@@ -154,28 +180,97 @@ __device__ __forceinline__ void decode_quarter(Stream& st, const uint8_t* lut, c
     }
 }
 
+// Starts the copy of the warp's 32 decoded rows (contiguous: 32 x 256 B from
+// `src`, the warp's first token) into its tile, rows kFullRow words apart
+// (cp.async, one commit group).  Copy i moves rows 2i and 2i + 1, lane l the
+// 16 bytes at (l & 15) * 16 of row 2i + (l >> 4), so every instruction reads
+// 512 contiguous bytes.  Rows from `valid` on are zero-filled (source size 0:
+// nothing is read).
+__device__ __forceinline__ void stage_rows_async(uint32_t tile, const uint16_t* src, int valid, int lane)
+{
+    const uint16_t* p = src + (lane >> 4) * 128 + (lane & 15) * 8;
+    uint32_t d = tile + (uint32_t)((lane >> 4) * kFullRow * 4 + (lane & 15) * 16);
+#pragma unroll 4
+    for (int r = lane >> 4; r < 32; r += 2) {
+        const bool ok = r < valid;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(ok ? p : src), "r"(ok ? 16u : 0u)
+                     : "memory");
+        p += 2 * 128;
+        d += 2 * kFullRow * 4;
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void stage_rows_wait()
+{
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// S += Q . K^T over dims 32 qd .. 32 qd + 31 of the warp's 32 staged tokens;
+// `stage_sh` addresses those dims of token 0, rows ROW words apart.
+template <int ROW = kStageRow>
+__device__ __forceinline__ void k_quarter_mma(float (&S)[4][4], const uint32_t* qrow, uint32_t stage_sh, int lane,
+                                              int qd)
+{
+    const int j0 = qd * 16;  // dims 32 qd.. as bf16 pairs
+    const uint32_t a00 = qrow[j0], a02 = qrow[j0 + 4], a10 = qrow[j0 + 8], a12 = qrow[j0 + 12];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        // matrices (lane >> 3): dims 0-7, 8-15, 16-23, 24-31 of tokens nt*8 + (lane & 7)
+        uint32_t bfr[4];
+        ldsm_x4(stage_sh + (uint32_t)(((nt * 8 + (lane & 7)) * ROW + (lane >> 3) * 4) * 4), bfr);
+        mma_bf16(S[nt], a00, 0u, a02, 0u, bfr[0], bfr[1]);
+        mma_bf16(S[nt], a10, 0u, a12, 0u, bfr[2], bfr[3]);
+    }
+}
+
+// acc[head][dims 32 qd ..] += P . V over the warp's 32 staged tokens.
+template <int G, int ROW = kStageRow>
+__device__ __forceinline__ void v_quarter_mma(float* s_acc, const uint32_t (&pa)[2][4], uint32_t stage_sh, int lane,
+                                              int gid, int tig, int qd)
+{
+#pragma unroll
+    for (int nd = 0; nd < 4; ++nd) {
+        // matrices (lane >> 3): tokens 0-7, 8-15, 16-23, 24-31 of dims nd*8..; lane l addresses token l
+        uint32_t bfr[4];
+        ldsm_x4_t(stage_sh + (uint32_t)((lane * ROW + nd * 4) * 4), bfr);
+        float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        mma_bf16(o, pa[0][0], pa[0][1], pa[0][2], pa[0][3], bfr[0], bfr[1]);
+        mma_bf16(o, pa[1][0], pa[1][1], pa[1][2], pa[1][3], bfr[2], bfr[3]);
+        if (gid < G) {
+            const int d = qd * 32 + nd * 8 + 2 * tig;
+            atomicAdd(&s_acc[gid * 128 + d], o[0] + o[2]);
+            atomicAdd(&s_acc[gid * 128 + d + 1], o[1] + o[3]);
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)
 {
     return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
 }
 
-template <int G>
+// STAGED = false: the CTA decodes its split's K and V blocks itself.
+// STAGED = true: the split's rows were decoded into A.kx / A.vx by the block
+// decoder just before (records already applied), and are read from there.
+template <int G, bool STAGED>
 __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_constant__ AttnArgs A)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t* smem = aligned_smem(smem_raw);
+    // unstaged only: tables, stream words, nibbles, per-token exchange
     uint8_t* s_lut = smem + kOffLut;
     float* s_Ct = reinterpret_cast<float*>(smem + kOffCt);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kOffWords);
     float* s_x = reinterpret_cast<float*>(smem + kOffX);
-    float* s_qf = reinterpret_cast<float*>(smem + kOffQf);
-    uint16_t* s_qb = reinterpret_cast<uint16_t*>(smem + kOffQb);
-    float* s_red = reinterpret_cast<float*>(smem + kOffRed);
-    float* s_acc = reinterpret_cast<float*>(smem + kOffAcc);
+    float* s_qf = reinterpret_cast<float*>(smem + (STAGED ? kSOffQf : kOffQf));
+    uint16_t* s_qb = reinterpret_cast<uint16_t*>(smem + (STAGED ? kSOffQb : kOffQb));
+    float* s_red = reinterpret_cast<float*>(smem + (STAGED ? kSOffRed : kOffRed));
+    float* s_acc = reinterpret_cast<float*>(smem + (STAGED ? kSOffAcc : kOffAcc));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;  // mma fragment coordinates
-    const int split = blockIdx.x, bh = blockIdx.y;
+    const int split = (STAGED ? A.split0 : 0) + (int)blockIdx.x, bh = blockIdx.y;
     const int b = bh / A.H, h = bh - b * A.H;
     const int Hq = A.H * G;
     const int tok0 = split * kAtThreads + warp * 32;  // first token of this warp
@@ -190,15 +285,19 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         s_qf[i] = bf16_bits_to_f32(v);
         s_acc[i] = 0.0f;
     }
-    stage_tables<kAtThreads>(A.ktb, s_lut, s_Ct, tid);
+    if constexpr (!STAGED) stage_tables<kAtThreads>(A.ktb, s_lut, s_Ct, tid);
     __syncthreads();
 
     uint32_t* ws = s_w + tid;
     uint32_t* nb = reinterpret_cast<uint32_t*>(smem + kOffNib) + tid;
-    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kOffStage) + warp * 32 * kStageRow;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kOffStage) + warp * 32 * kStageRow;  // unstaged
     uint32_t* row = stage + lane * kStageRow;
     const uint32_t stage_sh = (uint32_t)__cvta_generic_to_shared(stage);
     float* xw = s_x + warp * 32 * kHeads;
+    // staged: this warp's tile of whole rows, and this lane's row in it
+    const uint32_t tile_sh = (uint32_t)__cvta_generic_to_shared(smem + kSOffTile) + warp * 32 * kFullRow * 4;
+    const int64_t xoff = ((int64_t)bh * A.cstride + (tok0 - A.c0)) * 128;  // the warp's first row
+    const int valid = min(32, A.S - tok0);                                   // rows before the end (may be <= 0)
 
     // ---------------- K pass: S = Q K^T for the warp's 32 tokens
     float S[4][4];
@@ -206,7 +305,16 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) S[nt][e] = 0.0f;
-    {
+    if constexpr (STAGED) {
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(s_qb + gid * kQbRow) + tig;
+        stage_rows_async(tile_sh, valid > 0 ? A.kx + xoff : A.kx, valid, lane);
+        stage_rows_wait();
+        __syncwarp();
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) k_quarter_mma<kFullRow>(S, qrow, tile_sh + 64u * qd, lane, qd);
+        __syncwarp();  // every lane's K reads are done: the V rows go into the same tile during the softmax
+        stage_rows_async(tile_sh, valid > 0 ? A.vx + xoff : A.vx, valid, lane);
+    } else {
         uint4 q0, q1, q2, q3;
         const float s = load_block(A.kblk + blk * ECCO_BLOCK_BYTES, have, q0, q1, q2, q3, A.ktb->S_t);
         stage_words(ws, kAtStride, q0, q1, q2, q3);
@@ -219,16 +327,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         for (int qd = 0; qd < 4; ++qd) {
             decode_quarter(st, lut, ws, vp, row, nb, qd);
             __syncwarp();
-            const int j0 = qd * 16;  // dims 32 qd.. as bf16 pairs
-            const uint32_t a00 = qrow[j0], a02 = qrow[j0 + 4], a10 = qrow[j0 + 8], a12 = qrow[j0 + 12];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                // matrices (lane >> 3): dims 0-7, 8-15, 16-23, 24-31 of tokens nt*8 + (lane & 7)
-                uint32_t bfr[4];
-                ldsm_x4(stage_sh + (uint32_t)(((nt * 8 + (lane & 7)) * kStageRow + (lane >> 3) * 4) * 4), bfr);
-                mma_bf16(S[nt], a00, 0u, a02, 0u, bfr[0], bfr[1]);
-                mma_bf16(S[nt], a10, 0u, a12, 0u, bfr[2], bfr[3]);
-            }
+            k_quarter_mma(S, qrow, stage_sh, lane, qd);
             __syncwarp();
         }
         // outlier records: score += (new - old) * q[g][i], exchanged through shared memory
@@ -279,7 +378,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
             const float p = expf(S[nt][e] - M);  // exp(-inf) = 0 past the end
             S[nt][e] = p;
             sum += p;
-            xw[(nt * 8 + 2 * tig + e) * kHeads + gid] = p;  // p by token, for the V records
+            if constexpr (!STAGED) xw[(nt * 8 + 2 * tig + e) * kHeads + gid] = p;  // p by token, for the V records
         }
     sum += __shfl_xor_sync(0xffffffffu, sum, 1);
     sum += __shfl_xor_sync(0xffffffffu, sum, 2);
@@ -288,7 +387,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
     float L = 0.0f;
 #pragma unroll
     for (int w = 0; w < kAtWarps; ++w) L += s_red[kAtWarps * kHeads + w * kHeads + gid];
-    stage_tables<kAtThreads>(A.vtb, s_lut, s_Ct, tid);
+    if constexpr (!STAGED) stage_tables<kAtThreads>(A.vtb, s_lut, s_Ct, tid);
 
     // A fragments of P, k-step ks = tokens 16 ks + (0..15):
     // a0 / a2 (rows 0-7) = bf16(p), a1 / a3 (rows 8-15) = bf16(p - bf16(p))
@@ -307,7 +406,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
     __syncthreads();
 
     // ---------------- V pass: O = P V
-    {
+    if constexpr (STAGED) {
+        stage_rows_wait();
+        __syncwarp();  // other lanes' copies landed too
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) v_quarter_mma<G, kFullRow>(s_acc, pa, tile_sh + 64u * qd, lane, gid, tig, qd);
+    } else {
         uint4 q0, q1, q2, q3;
         const float s = load_block(A.vblk + blk * ECCO_BLOCK_BYTES, have, q0, q1, q2, q3, A.vtb->S_t);
         stage_words(ws, kAtStride, q0, q1, q2, q3);
@@ -318,20 +422,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         for (int qd = 0; qd < 4; ++qd) {
             decode_quarter(st, lut, ws, vp, row, nb, qd);
             __syncwarp();
-#pragma unroll
-            for (int nd = 0; nd < 4; ++nd) {
-                // matrices (lane >> 3): tokens 0-7, 8-15, 16-23, 24-31 of dims nd*8..; lane l addresses token l
-                uint32_t bfr[4];
-                ldsm_x4_t(stage_sh + (uint32_t)((lane * kStageRow + nd * 4) * 4), bfr);
-                float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                mma_bf16(o, pa[0][0], pa[0][1], pa[0][2], pa[0][3], bfr[0], bfr[1]);
-                mma_bf16(o, pa[1][0], pa[1][1], pa[1][2], pa[1][3], bfr[2], bfr[3]);
-                if (gid < G) {
-                    const int d = qd * 32 + nd * 8 + 2 * tig;
-                    atomicAdd(&s_acc[gid * 128 + d], o[0] + o[2]);
-                    atomicAdd(&s_acc[gid * 128 + d + 1], o[1] + o[3]);
-                }
-            }
+            v_quarter_mma<G>(s_acc, pa, stage_sh, lane, gid, tig, qd);
             __syncwarp();
         }
         const float* pt = xw + lane * kHeads;  // this token's p per head
@@ -371,22 +462,61 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict
     out[(int64_t)bq * 128 + d] = acc / L;
 }
 
-template <int G>
-cudaError_t run_attn(const AttnArgs& A, int B, cudaStream_t s, float* out)
+template <int G, bool STAGED>
+cudaError_t configure_attn()
 {
     static int configured = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured != dev) {
-        cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kAttnSmem);
+        cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<G, STAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(STAGED ? kAttnSmemStaged : kAttnSmem));
         if (e != cudaSuccess) return e;
         configured = dev;
     }
-    dim3 grid((unsigned)A.splits, (unsigned)(B * A.H));
-    attn_split_kernel<G><<<grid, kAtThreads, kAttnSmem, s>>>(A);
-    cudaError_t e = cudaGetLastError();
+    return cudaSuccess;
+}
+
+template <int G>
+cudaError_t run_attn(const AttnArgs& A, int B, cudaStream_t s, float* out)
+{
+    cudaError_t e = configure_attn<G, false>();
     if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)A.splits, (unsigned)(B * A.H));
+    attn_split_kernel<G, false><<<grid, kAtThreads, kAttnSmem, s>>>(A);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_merge_kernel<<<B * A.H * G, 128, 0, s>>>(A.ws, A.splits, out);
+    return cudaGetLastError();
+}
+
+// Staged: per chunk of tokens, the block decoder writes the chunk's K and V
+// rows to the scratch (one two-segment launch), then the split kernel reads
+// them; the merge runs once over all splits.
+template <int G>
+cudaError_t run_attn_staged(AttnArgs A, int B, const ecco_tables* kt, const ecco_tables* vt, uint16_t* scratch,
+                            cudaStream_t s, float* out)
+{
+    cudaError_t e = configure_attn<G, true>();
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)B * A.H, C = staged_chunk_tokens(B, A.H, A.S);
+    A.kx = scratch;
+    A.vx = scratch + rows * C * kG;
+    A.cstride = C;
+    for (int64_t c0 = 0; c0 < A.S; c0 += C) {
+        const int64_t cn = (A.S - c0 < C) ? A.S - c0 : C;
+        ecco_segment seg[2];
+        seg[0] = ecco_segment{kt, A.kblk, scratch, ecco_desc{rows, cn, A.s_cap, C, c0, 0}};
+        seg[1] = ecco_segment{vt, A.vblk, scratch + rows * C * kG, ecco_desc{rows, cn, A.s_cap, C, c0, 0}};
+        e = launch_decode_multi(seg, 2, s);
+        if (e != cudaSuccess) return e;
+        A.c0 = c0;
+        A.split0 = (int)(c0 / kAtThreads);
+        dim3 grid((unsigned)((cn + kAtThreads - 1) / kAtThreads), (unsigned)rows);
+        attn_split_kernel<G, true><<<grid, kAtThreads, kAttnSmemStaged, s>>>(A);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     attn_merge_kernel<<<B * A.H * G, 128, 0, s>>>(A.ws, A.splits, out);
     return cudaGetLastError();
 }
@@ -395,11 +525,20 @@ cudaError_t run_attn(const AttnArgs& A, int B, cudaStream_t s, float* out)
 
 int attention_splits(int seq_len) { return (seq_len + kAtThreads - 1) / kAtThreads; }
 
+int64_t staged_chunk_tokens(int B, int H, int seq_len)
+{
+    const int64_t per_token = (int64_t)B * H * 2 * kG * 2;  // K and V bf16 rows of one token position
+    int64_t c = kStagedScratchBytes / per_token / kAtThreads * kAtThreads;
+    const int64_t whole = ((int64_t)seq_len + kAtThreads - 1) / kAtThreads * kAtThreads;
+    if (c < kAtThreads) c = kAtThreads;
+    return c < whole ? c : whole;
+}
+
 cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
                              const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
                              const uint16_t* q, float scale, float* out, float* ws, cudaStream_t s)
 {
-    AttnArgs A{kt->d, vt->d, kblk, vblk, s_cap, H, G, S, attention_splits(S), q, scale, ws};
+    AttnArgs A{kt->d, vt->d, kblk, vblk, s_cap, H, G, S, attention_splits(S), q, scale, ws, nullptr, nullptr, 0, 0, 0};
     switch (G) {
         case 1: return run_attn<1>(A, B, s, out);
         case 2: return run_attn<2>(A, B, s, out);
@@ -409,6 +548,25 @@ cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const
         case 6: return run_attn<6>(A, B, s, out);
         case 7: return run_attn<7>(A, B, s, out);
         case 8: return run_attn<8>(A, B, s, out);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_attention_staged(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                                    const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
+                                    const uint16_t* q, float scale, float* out, float* ws, uint16_t* scratch,
+                                    cudaStream_t s)
+{
+    AttnArgs A{kt->d, vt->d, kblk, vblk, s_cap, H, G, S, attention_splits(S), q, scale, ws, nullptr, nullptr, 0, 0, 0};
+    switch (G) {
+        case 1: return run_attn_staged<1>(A, B, kt, vt, scratch, s, out);
+        case 2: return run_attn_staged<2>(A, B, kt, vt, scratch, s, out);
+        case 3: return run_attn_staged<3>(A, B, kt, vt, scratch, s, out);
+        case 4: return run_attn_staged<4>(A, B, kt, vt, scratch, s, out);
+        case 5: return run_attn_staged<5>(A, B, kt, vt, scratch, s, out);
+        case 6: return run_attn_staged<6>(A, B, kt, vt, scratch, s, out);
+        case 7: return run_attn_staged<7>(A, B, kt, vt, scratch, s, out);
+        case 8: return run_attn_staged<8>(A, B, kt, vt, scratch, s, out);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -161,15 +161,15 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
             }
 
             if (st.room >= 0) {  // unclipped: outlier records follow the codewords
-                // The walk ended exactly at the first record, so the stream
-                // window reads them in order.  q / 127 is divided here (an
-                // ALU sequence) rather than looked up: the kernel is bound by
-                // the L1 data path, which a table gather would load further.
+                // Each record is read at its own offset (independent loads,
+                // no chain through the stream window).  q / 127 is divided
+                // here (an ALU sequence) rather than looked up: the kernel is
+                // bound by the L1 data path, which a table gather would load
+                // further.
                 const int n = min(kMaxRec, st.room / kRecBits);
+                const int at0 = kBlockBits - st.room;
                 for (int k = 0; k < n; ++k) {
-                    refill(st, ws, kWordStride);
-                    const uint32_t rec = __funnelshift_r(st.lo, st.hi, st.b);
-                    st.b += kRecBits;
+                    const uint32_t rec = read_record(ws, kWordStride, at0 + k * kRecBits);
                     const int i = (int)(rec & (uint32_t)(G - 1));  // the 7-bit index, modulo G
                     const float o = __fdiv_rn((float)(int)(int8_t)(uint8_t)(rec >> 7), 127.0f);
                     const uint16_t v = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));

@@ -84,6 +84,14 @@ int attention_splits(int seq_len);
 cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
                              const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
                              const uint16_t* q, float scale, float* out, float* ws, cudaStream_t s);
+// Staged attention: chunks of staged_chunk_tokens() tokens decoded into
+// `scratch` ([2][B*H][chunk][128] bf16) by the block decoder, then the split
+// kernel over the decoded rows.
+int64_t staged_chunk_tokens(int B, int H, int seq_len);
+cudaError_t launch_attention_staged(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                                    const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
+                                    const uint16_t* q, float scale, float* out, float* ws, uint16_t* scratch,
+                                    cudaStream_t s);
 
 // Table learner (offline): the blob of one tensor from a device bf16 sample.
 cudaError_t learn_tables(const uint16_t* x, int64_t n_groups, int G, int npat, uint64_t seed, uint8_t* blob,

@@ -217,6 +217,29 @@ int ecco_decode_attention(const ecco_tables* k_tables, const ecco_tables* v_tabl
                           float scale, float* out, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* The same attention (same arguments, result and tolerance), computed in
+ * stages: for each chunk of tokens the block decoder (ecco_decode_multi's
+ * kernel) writes the chunk's decoded K and V rows to a scratch inside the
+ * workspace, then a split kernel reads them back with coalesced copies.  A
+ * chunk holds whole 512-token splits, and its rows (2 x batch x kv_heads x
+ * chunk x 256 B) stay within 1 GiB, so most caches run as one chunk.  The
+ * decoded rows cross HBM once each way; in exchange the decode runs at the
+ * standalone decoder's occupancy, which the single fused kernel cannot reach
+ * (its tables, stream words and tiles leave it half the resident warps).  The
+ * review page's point that compression speeds up the decode-phase reads of
+ * the cache ("If this is right", Fig. 11 caption) holds for both: the
+ * compressed blocks are what is read from the cache.
+ *   workspace  at least ecco_decode_attention_staged_workspace_bytes(...)
+ *              bytes, 4-byte aligned, caller-owned; it holds the per-split
+ *              partial results and the chunk scratch (no initial contents).
+ * Errors and the other arguments as for ecco_decode_attention. */
+size_t ecco_decode_attention_staged_workspace_bytes(int batch, int kv_heads, int group, int seq_len);
+int ecco_decode_attention_staged(const ecco_tables* k_tables, const ecco_tables* v_tables,
+                                 const uint8_t* k_blocks, const uint8_t* v_blocks, int64_t seq_capacity,
+                                 int batch, int kv_heads, int group, int seq_len, const uint16_t* q_bf16,
+                                 float scale, float* out, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* ecco_decode_attention with its workspace in static device memory: a
  * file-scope __device__ array of ECCO_ATTENTION_STATIC_WS_BYTES per device
  * inside the library, so the call allocates nothing and takes no workspace

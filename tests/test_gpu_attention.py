@@ -1,4 +1,7 @@
-"""Fused decode + decode-phase attention (CUDA, through the C ABI) vs the oracle.
+"""Decode-phase attention over compressed K and V (CUDA, through the C ABI) vs
+the oracle, for both entry points: ecco_decode_attention (the blocks decoded
+inside the attention kernel) and ecco_decode_attention_staged (each chunk of
+tokens decoded by the block decoder into a scratch, then attended).
 
 The oracle decodes the K and V blocks and applies softmax attention in
 float64.  The kernel decodes the same blocks bit-exactly (the block decoder's
@@ -44,11 +47,15 @@ def check(out, ref, aw):
                            f"{(err - RTOL * aw).max():.3e}")
 
 
-def run(kt, vt, kb, vb, q, seq_len, scale, ws=None):
+PATHS = {"fused": (ecco.decode_attention, ecco.attention_workspace_bytes),
+         "staged": (ecco.decode_attention_staged, ecco.attention_staged_workspace_bytes)}
+
+
+def run(kt, vt, kb, vb, q, seq_len, scale, ws=None, path="fused"):
     B, H, S, _ = kb.shape
-    return ecco.decode_attention(torch.from_numpy(kb).to(DEV), torch.from_numpy(vb).to(DEV),
-                                 ecco.Tables(kt, DEV), ecco.Tables(vt, DEV), to_dev_bf16(q), seq_len,
-                                 scale, workspace=ws).cpu().numpy()
+    return PATHS[path][0](torch.from_numpy(kb).to(DEV), torch.from_numpy(vb).to(DEV),
+                          ecco.Tables(kt, DEV), ecco.Tables(vt, DEV), to_dev_bf16(q), seq_len,
+                          scale, workspace=ws).cpu().numpy()
 
 
 CASES = [
@@ -64,8 +71,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["fused", "staged"])
 @pytest.mark.parametrize("B,H,G,S_cap,n,ktn,vtn,kk,vk", CASES)
-def test_attention_matches_oracle(B, H, G, S_cap, n, ktn, vtn, kk, vk):
+def test_attention_matches_oracle(B, H, G, S_cap, n, ktn, vtn, kk, vk, path):
     kt, vt = table_set(ktn), table_set(vtn)
     kb, _ = oracle.encode(kt, inputs(kk, B * H * S_cap, seed=S_cap), nthreads=8)
     vb, _ = oracle.encode(vt, inputs(vk, B * H * S_cap, seed=S_cap + 1), nthreads=8)
@@ -74,11 +82,29 @@ def test_attention_matches_oracle(B, H, G, S_cap, n, ktn, vtn, kk, vk):
     q = q_bits(B, H * G, seed=n)
     scale = 1.0 / np.sqrt(128.0)
     ref, aw = oracle.attention(kt, vt, kb, vb, q, n, scale)
-    out = run(kt, vt, kb, vb, q, n, scale)
+    out = run(kt, vt, kb, vb, q, n, scale, path=path)
     check(out, ref, aw)
 
 
-def test_blocks_past_seq_len_are_never_used():
+def test_staged_chunks():
+    """4096 (batch, KV head) rows make the staged chunk 512 tokens (1 GiB of
+    decoded rows), so 1237 tokens run as chunks of 512, 512 and 213 tokens
+    through the same scratch."""
+    B, H, G, S_cap, n = 512, 8, 1, 1240, 1237
+    assert _lib.load().ecco_decode_attention_staged_workspace_bytes(B, H, G, n) == (
+        4 * 130 * B * H * G * 3 + 256 + 2 * B * H * 512 * 256)
+    kt, vt = table_set("learned_kv"), table_set("random2")
+    rng = np.random.default_rng(31)  # every 64-byte pattern is a block (clips, records, null scales)
+    kb = rng.integers(0, 256, (B, H, S_cap, 64), dtype=np.uint8)
+    vb = rng.integers(0, 256, (B, H, S_cap, 64), dtype=np.uint8)
+    q = q_bits(B, H * G, seed=33)
+    ref, aw = oracle.attention(kt, vt, kb, vb, q, n, 1e-3, nthreads=8)
+    assert np.isfinite(ref).all()
+    check(run(kt, vt, kb, vb, q, n, 1e-3, path="staged"), ref, aw)
+
+
+@pytest.mark.parametrize("path", ["fused", "staged"])
+def test_blocks_past_seq_len_are_never_used(path):
     """Garbage after seq_len (random bytes) must not change the result."""
     B, H, G, S_cap, n = 1, 2, 4, 1500, 1111
     kt = vt = table_set("learned_kv")
@@ -91,20 +117,22 @@ def test_blocks_past_seq_len_are_never_used():
     vb2[:, :, n:] = rng.integers(0, 256, vb2[:, :, n:].shape, dtype=np.uint8)
     q = q_bits(B, H * G, seed=4)
     ref, aw = oracle.attention(kt, vt, kb, vb, q, n, 0.1)
-    check(run(kt, vt, kb2, vb2, q, n, 0.1), ref, aw)
+    check(run(kt, vt, kb2, vb2, q, n, 0.1, path=path), ref, aw)
 
 
-def test_workspace_reused_across_two_calls():
+@pytest.mark.parametrize("path", ["fused", "staged"])
+def test_workspace_reused_across_two_calls(path):
     B, H, G, S_cap, n = 2, 2, 4, 1024, 1000
     kt = vt = table_set("learned_kv")
     kb, _ = oracle.encode(kt, inputs("kv", B * H * S_cap, seed=5), nthreads=8)
     vb, _ = oracle.encode(vt, inputs("kv", B * H * S_cap, seed=6), nthreads=8)
     kb, vb = kb.reshape(B, H, S_cap, 64), vb.reshape(B, H, S_cap, 64)
-    ws = torch.empty(ecco.attention_workspace_bytes(B, H, G, n), dtype=torch.uint8, device=DEV)
+    # garbage in the workspace (partials and scratch) must not matter
+    ws = torch.full((PATHS[path][1](B, H, G, n),), 0xff, dtype=torch.uint8, device=DEV)
     for seed in (7, 8):
         q = q_bits(B, H * G, seed=seed)
         ref, aw = oracle.attention(kt, vt, kb, vb, q, n, 0.09)
-        check(run(kt, vt, kb, vb, q, n, 0.09, ws=ws), ref, aw)
+        check(run(kt, vt, kb, vb, q, n, 0.09, ws=ws, path=path), ref, aw)
 
 
 def test_full_size_kv_cache_attention_sampled():
@@ -122,6 +150,8 @@ def test_full_size_kv_cache_attention_sampled():
     q = q_bits(B, H * G, seed=21)
     scale = 1.0 / np.sqrt(128.0)
     out = ecco.decode_attention(kb, vb, tk, tv, to_dev_bf16(q), S, scale).cpu().numpy()
+    # staged: 64 rows make 1024-token chunks, so four chunks through the scratch
+    outs = ecco.decode_attention_staged(kb, vb, tk, tv, to_dev_bf16(q), S, scale).cpu().numpy()
     for b, h in ((0, 0), (3, 5), (7, 7), (5, 2)):
         kbo, _ = oracle.encode(kt, W.bf16_bits(K[b, h]), nthreads=8)
         vbo, _ = oracle.encode(vt, W.bf16_bits(V[b, h]), nthreads=8)
@@ -130,6 +160,7 @@ def test_full_size_kv_cache_attention_sampled():
         ref, aw = oracle.attention(kt, vt, kbo.reshape(1, 1, S, 64), vbo.reshape(1, 1, S, 64),
                                    q[b:b + 1, h * G:(h + 1) * G], S, scale)
         check(out[b:b + 1, h * G:(h + 1) * G], ref, aw)
+        check(outs[b:b + 1, h * G:(h + 1) * G], ref, aw)
 
 
 def test_attention_argument_errors():
@@ -155,6 +186,21 @@ def test_attention_argument_errors():
     assert call(ws_bytes=4 * 130 * 4 - 1) == _lib.ECCO_ERR_ARG
     assert call(kptr=kb.data_ptr() + 8) == _lib.ECCO_ERR_ALIGN
 
+    need = lib.ecco_decode_attention_staged_workspace_bytes(1, 1, 4, 64)
+    wss = torch.empty(need, dtype=torch.uint8, device=DEV)
+
+    def staged(kptr=kb.data_ptr(), group=4, n=64, ws_bytes=need):
+        return lib.ecco_decode_attention_staged(t.handle, t.handle, P(kptr), P(kb.data_ptr()), 64, 1, 1, group,
+                                                n, P(q.data_ptr()), 1.0, P(out.data_ptr()), P(wss.data_ptr()),
+                                                ws_bytes, None)
+
+    assert staged() == _lib.ECCO_OK
+    torch.cuda.synchronize()
+    assert staged(group=9) == _lib.ECCO_ERR_ARG
+    assert staged(n=65) == _lib.ECCO_ERR_ARG
+    assert staged(ws_bytes=need - 1) == _lib.ECCO_ERR_ARG
+    assert staged(kptr=kb.data_ptr() + 8) == _lib.ECCO_ERR_ALIGN
+
 
 def test_attention_on_garbage_blocks():
     """Random K and V blocks (clipped streams, duplicate record indexes, null
@@ -169,3 +215,4 @@ def test_attention_on_garbage_blocks():
     ref, aw = oracle.attention(kt, vt, kb, vb, q, n, scale)
     assert np.isfinite(ref).all()
     check(run(kt, vt, kb, vb, q, n, scale), ref, aw)
+    check(run(kt, vt, kb, vb, q, n, scale, path="staged"), ref, aw)
