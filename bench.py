@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ecco", choices=["ecco", "reference"])
     ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select", "act"])
+    ap.add_argument("--attention", default="staged", choices=["staged", "fused"],
+                    help="attn workload: decode_attention_staged (default) or the single fused kernel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
@@ -537,6 +539,7 @@ class AttnWorkload(Workload):
     tokens, the blocks decoded inside the attention kernel."""
     name = "attn"
     B, H, S, D, G = 8, 8, 4096, 128, 4
+    path = "staged"  # or "fused": the single kernel that decodes inside the attention
 
     def __init__(self, dev, seed_offset=0):
         import torch
@@ -544,10 +547,12 @@ class AttnWorkload(Workload):
         import entropy_coded_kv_b200 as ecco
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev = torch, ecco, dev
+        how = ("staged decode+attention over all 4096 tokens (block decoder into a workspace scratch, then "
+               "the split kernel)" if self.path == "staged" else
+               "fused decode+attention over all 4096 tokens (one kernel decodes and attends)")
         self.desc = ("decode-phase attention over a compressed Llama-3-8B-shaped layer KV cache: K, V "
                      "[8, 8, 4096, 128] as 64-byte blocks, 32 query heads (group 4); a step appends one "
-                     "token's K and V (128 groups) and runs staged decode+attention over all 4096 tokens "
-                     "(block decoder into a workspace scratch, then the split kernel)")
+                     "token's K and V (128 groups) and runs " + how)
         K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
         Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
         self.tables = [ecco.Tables(learn_tables(Kc, seed=0), dev), ecco.Tables(learn_tables(Vc, seed=0), dev)]
@@ -562,12 +567,16 @@ class AttnWorkload(Workload):
         g = torch.Generator(device=dev).manual_seed(77 + seed_offset)
         self.q = torch.randn(self.B, self.H * self.G, self.D, generator=g, device=dev).to(torch.bfloat16)
         self.out = torch.empty(self.B, self.H * self.G, self.D, dtype=torch.float32, device=dev)
-        self.ws = torch.empty(ecco.attention_staged_workspace_bytes(self.B, self.H, self.G, self.S),
-                              dtype=torch.uint8, device=dev)
+        staged = self.path == "staged"
+        ws_bytes = ecco.attention_staged_workspace_bytes if staged else ecco.attention_workspace_bytes
+        self.ws = torch.empty(ws_bytes(self.B, self.H, self.G, self.S), dtype=torch.uint8, device=dev)
+        self.attend = ecco.decode_attention_staged if staged else ecco.decode_attention
         self.scale = 1.0 / self.D ** 0.5
-        # append (one multi-segment launch); one chunk: decode (K and V in one launch), split kernel; merge
-        self.launches_per_step = 4
-        self.api = "entropy_coded_kv_b200.encode_multi/decode_attention_staged (C ABI) with pinned host buffers"
+        # append (one multi-segment launch); staged, one chunk: decode (K and V in one launch) and the
+        # split kernel; fused: the split kernel; then the merge
+        self.launches_per_step = 4 if staged else 3
+        self.api = (f"entropy_coded_kv_b200.encode_multi/{self.attend.__name__} (C ABI) with pinned host "
+                    "buffers")
         self.att_ms = []
 
     def bytes_decoded(self):  # bf16 K and V bytes the step decodes
@@ -580,8 +589,8 @@ class AttnWorkload(Workload):
         return 1.0 / 64
 
     def _attend(self, q):
-        return self.ecco.decode_attention_staged(self.blocks[0], self.blocks[1], self.tables[0], self.tables[1], q,
-                                                 self.S, self.scale, out=self.out, workspace=self.ws)
+        return self.attend(self.blocks[0], self.blocks[1], self.tables[0], self.tables[1], q, self.S, self.scale,
+                           out=self.out, workspace=self.ws)
 
     def step(self, record=False):
         self.ecco.encode_multi(self.app)
@@ -598,7 +607,9 @@ class AttnWorkload(Workload):
         self.torch.cuda.synchronize()
         ms = [a.elapsed_time(b) for a, b in self.att_ms]
         nbytes = 2 * self.n * 64 + self.q.numel() * 2 + self.out.numel() * 4
-        return "decode_kernel+attn_split_kernel+attn_merge_kernel", nbytes, ms
+        kernels = "decode_kernel+attn_split_kernel+attn_merge_kernel" if self.path == "staged" else \
+            "attn_split_kernel+attn_merge_kernel"
+        return kernels, nbytes, ms
 
     def e2e_setup(self):
         torch = self.torch
@@ -875,6 +886,7 @@ def main():
         dist.barrier()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    AttnWorkload.path = args.attention
     wl = WORKLOADS[args.workload](dev, seed_offset=0)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
@@ -976,6 +988,7 @@ KERNEL_SOURCES = {
     "decode_kernel<G=64>": ["ecco_decode.cu", "ecco_block.cuh"],
     "encode_kernel<.,SEL=1>": ["ecco_encode.cu"],
     "decode_kernel+attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_decode.cu", "ecco_block.cuh"],
+    "attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_block.cuh"],
 }
 
 
@@ -1013,6 +1026,7 @@ def run_reference(args, world):
     if dev is None:
         print(json.dumps({"impl": "reference", "unavailable": "workload inputs are generated on a CUDA device"}))
         return
+    AttnWorkload.path = args.attention
     wl = WORKLOADS[args.workload](dev)
     cores = os.cpu_count() or 1
     sample = wl.cpu_sample(wl.cpu_frac())
