@@ -1,0 +1,68 @@
+"""Host-side logic of bench.py (no GPU): the committed DRAM-traffic entries and
+their source hashes, the peak lookup, and the reference arm's line on a
+machine without a CUDA device."""
+from __future__ import annotations
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_every_traffic_entry_names_a_known_kernel_and_its_capture():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        entries = json.load(f)["entries"]
+    assert entries
+    for key, e in entries.items():
+        workload, kernel = key.split(":", 1)
+        assert workload in bench.WORKLOADS, key
+        assert kernel.split(" ")[0] in bench.KERNEL_SOURCES, key
+        assert os.path.exists(os.path.join(ROOT, e["capture"])), key
+        assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"], key
+
+
+def test_traffic_is_reported_only_while_the_sources_are_unchanged(monkeypatch):
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        entries = json.load(f)["entries"]
+    key = "kv:decode_kernel"
+    e = entries[key]
+    monkeypatch.setattr(bench, "source_hash", lambda files: e["source_hash"])
+    assert bench.traffic_for("kv", "decode_kernel") == e["dram_bytes_per_launch"]
+    monkeypatch.setattr(bench, "source_hash", lambda files: "0" * 16)
+    assert bench.traffic_for("kv", "decode_kernel") is None
+    assert bench.traffic_for("kv", "no_such_kernel") is None
+
+
+def test_source_hash_covers_every_listed_file():
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.exists(os.path.join(ROOT, "entropy_coded_kv_b200", "csrc", f)), (kernel, f)
+        assert len(bench.source_hash(files)) == 16
+
+
+def test_peak_comes_from_the_measured_file_when_present():
+    value, source = bench.peaks()
+    if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            assert value == float(json.load(f)["hbm_gbs"]) and source == "measured"
+    else:
+        assert (value, source) == (bench.FALLBACK_HBM_GBS, "fallback")
+
+
+def test_attention_workload_defaults_to_the_staged_path():
+    assert bench.AttnWorkload.path == "staged"
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device line")
+def test_reference_arm_without_a_device_prints_its_unavailable_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and "unavailable" in line
