@@ -190,8 +190,10 @@ def decode_attention_staged(k_blocks: torch.Tensor, v_blocks: torch.Tensor, k_ta
                             q: torch.Tensor, seq_len: int, scale: float, out: torch.Tensor | None = None,
                             workspace: torch.Tensor | None = None) -> torch.Tensor:
     """decode_attention computed in stages: each chunk of tokens is decoded by
-    the block decoder into a scratch in the workspace (sized to stay in L2),
-    then attended.  Same arguments and result."""
+    the block decoder into a scratch in the workspace, then attended.  Same
+    arguments and result.  The workspace holds a chunk's decoded K and V rows
+    (up to 1 GiB, attention_staged_workspace_bytes); pass one to reuse it
+    across calls."""
     return _attention("ecco_decode_attention_staged", attention_staged_workspace_bytes, k_blocks, v_blocks,
                       k_tables, v_tables, q, seq_len, scale, out, workspace)
 
