@@ -85,8 +85,12 @@ cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const
                              const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
                              const uint16_t* q, float scale, float* out, float* ws, cudaStream_t s);
 // Staged attention: chunks of staged_chunk_tokens() tokens decoded into
-// `scratch` ([2][B*H][chunk][128] bf16) by the block decoder, then the split
-// kernel over the decoded rows.
+// `scratch` ([2][B*H][chunk][128] bf16) by the block decoder, then a split
+// kernel without tables copies whole decoded rows into shared memory
+// (cp.async) and runs the same products and softmax as launch_attention's
+// kernel.  On B200 it is the faster of the two: the fused kernel's tables,
+// stream words and tiles leave it half the decoder's resident warps, so its
+// serial walk shows through.
 int64_t staged_chunk_tokens(int B, int H, int seq_len);
 cudaError_t launch_attention_staged(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
                                     const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
