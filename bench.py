@@ -1,15 +1,17 @@
 #!/usr/bin/env python
 """Throughput of the Ecco block codec on one or more B200s (one process per GPU).
 
-Default workload (`--workload kv`): one Llama-3-8B-shaped layer of KV cache,
-K and V each [8, 8, 4096, 128] bf16.  A step encodes the last 64 tokens of K
-and V (8,192 groups, written into the compressed cache) and decodes the whole
-compressed cache back to bf16 (524,288 blocks); K and V go through one
-multi-segment launch each way (`encode_multi`, `decode_multi`).  Other
-workloads: `c1` (256 x 1024 matrix, encode + decode), `mlp` (14336 x 4096
-weight: encode, decode, fused decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights,
-encode and decode of the whole set), `longctx` (32 layers x K,V x
-[1, 8, 131072, 128]: full streaming decode plus a one-token append per layer),
+Default workload (`--workload longctx`, the largest configuration): a
+32-layer long-context KV cache, K and V of every layer [1, 8, 131072, 128]
+bf16 (17.2 GB).  A step appends one token to every layer's K and V (512
+groups, encoded into the compressed cache) and decodes the whole compressed
+cache back to bf16 (67,108,864 blocks); each direction is one multi-segment
+call (`encode_multi`, `decode_multi`: 64 tensors in one launch).  Other
+workloads: `kv` (one Llama-3-8B-shaped layer, K and V [8, 8, 4096, 128]:
+encode of the last 64 tokens + decode of the whole cache), `c1` (256 x 1024
+matrix, encode + decode), `mlp` (14336 x 4096 weight: encode, decode, fused
+decode+GEMV at batch 1 and 16), `model` (32 layers x 7 weights, encode and
+decode of the whole set),
 `attn` (one-token append + staged decode+attention over the compressed cache of
 the `kv` layer, 32 query heads), `select` (encode of the `kv` layer with
 full-MSE pattern selection, plus a quality study of min/max vs full-MSE
@@ -36,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decoded GB/s (bf16 out) & encode GB/s, % of HBM roofline, bit-exact vs oracle"
+TABLE_BLOB_BYTES = 7952  # one tensor's stored tables: S_t, 64 x 15 centroids, 64 x 4 x 16 code lengths
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -45,7 +48,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ecco", choices=["ecco", "reference"])
-    ap.add_argument("--workload", default="kv", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select", "act"])
+    ap.add_argument("--workload", default="longctx", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select", "act"])
     ap.add_argument("--attention", default="staged", choices=["staged", "fused"],
                     help="attn workload: decode_attention_staged (default) or the single fused kernel")
     ap.add_argument("--no-e2e", action="store_true")
@@ -132,6 +135,28 @@ class Workload:
     name = ""
     desc = ""
     launches_per_step = 0
+    stats = None       # ecco_stats counters of one encode of the whole workload (setup, untimed)
+    n_tensors = 1      # tensors with their own table blob
+    group = 128        # values per group
+
+    def stats_summary(self):
+        """Clipping, padding and compression of the workload's blocks: the
+        review page's Fig. 10 (padding and clipping ratios) and "Core claim"
+        (memory reduction) quantities, from the encoder's own counters."""
+        if not self.stats:
+            return None
+        st = self.stats
+        n = max(1, st["n_groups"])
+        raw = st["n_groups"] * self.group * 2
+        blocks = st["n_groups"] * 64
+        tables = self.n_tensors * TABLE_BLOB_BYTES
+        return {"groups": st["n_groups"], "clip_ratio": round(st["n_clipped"] / n, 5),
+                "pad_ratio": round(st["n_padded"] / n, 5), "records_per_block": round(st["n_records"] / n, 4),
+                "payload_bits_per_block": round(st["payload_bits"] / n, 2),
+                "zero_blocks": st["n_zero"], "nonfinite_values": st["n_nonfinite"],
+                "compression_ratio": round(raw / blocks, 4),
+                "compression_ratio_with_tables": round(raw / (blocks + tables), 4),
+                "table_blob_bytes": TABLE_BLOB_BYTES, "tensors": self.n_tensors}
 
     def bytes_decoded(self) -> int:      # bf16 bytes written by decode per step
         return 0
@@ -143,6 +168,57 @@ class Workload:
         return 0
 
 
+class LayerStream:
+    """End-to-end leg of the two large workloads, streamed layer by layer.
+
+    Per layer: host-to-device copies of that layer's inputs (from pinned host
+    memory) on one stream, the library calls on the current stream once those
+    copies landed, device-to-host copies of that layer's results on a third
+    stream once the calls finished.  Copies of one layer overlap the calls of
+    the next.  Inputs come from pinned host copies of the whole step's inputs;
+    results go to two pinned staging buffers used by alternate layers (the host
+    does not read them while the step is timed), so every input byte crosses
+    to the device and every result byte crosses back once per step."""
+
+    def __init__(self, torch, dev, layers):
+        """layers: [(ins, run, outs)]: ins = [(host pinned, device)] pairs,
+        run() enqueues the layer's library calls on the current stream, outs =
+        device tensors to copy back."""
+        self.torch, self.layers = torch, layers
+        self.s_in, self.s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        most = max(sum(t.numel() * t.element_size() for t in outs) for _, _, outs in layers)
+        self.stage = [torch.empty(most, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self.h2d = sum(h.numel() * h.element_size() for ins, _, _ in layers for h, _ in ins)
+        self.d2h = sum(t.numel() * t.element_size() for _, _, outs in layers for t in outs)
+
+    def step(self):
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        go = torch.cuda.Event()
+        go.record(main)
+        self.s_in.wait_event(go)
+        for li, (ins, run, outs) in enumerate(self.layers):
+            with torch.cuda.stream(self.s_in):
+                for h, d in ins:
+                    d.copy_(h, non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(self.s_in)
+            main.wait_event(landed)
+            run()
+            ran = torch.cuda.Event()
+            ran.record(main)
+            self.s_out.wait_event(ran)
+            with torch.cuda.stream(self.s_out):
+                st, off = self.stage[li % 2], 0
+                for t in outs:
+                    nb = t.numel() * t.element_size()
+                    st[off:off + nb].copy_(t.reshape(-1).view(torch.uint8), non_blocking=True)
+                    off += nb
+        done = torch.cuda.Event()
+        done.record(self.s_out)
+        main.wait_event(done)
+
+
 def _events(torch):
     return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
@@ -150,6 +226,8 @@ def _events(torch):
 class KVWorkload(Workload):
     """One layer of KV cache: encode 64 new tokens, decode the whole cache."""
     name = "kv"
+    desc = ("Llama-3-8B-shaped one-layer KV cache, K and V each [8, 8, 4096, 128] bf16: "
+            "encode the last 64 tokens (8,192 groups) + decode the full cache (524,288 blocks)")
     B, H, S, D, T = 8, 8, 4096, 128, 64
 
     def __init__(self, dev, seed_offset=0):
@@ -158,15 +236,15 @@ class KVWorkload(Workload):
         import entropy_coded_kv_b200 as ecco
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        self.desc = ("Llama-3-8B-shaped one-layer KV cache, K and V each [8, 8, 4096, 128] bf16: "
-                     "encode the last 64 tokens (8,192 groups) + decode the full cache (524,288 blocks)")
         K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
         Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
         self.tables = [ecco.Tables(learn_tables(Kc, seed=0), dev), ecco.Tables(learn_tables(Vc, seed=0), dev)]
         self.rows = self.B * self.H
         self.n = self.rows * self.S
         self.caches = [K, V]
-        self.blocks = [ecco.encode(K, self.tables[0]), ecco.encode(V, self.tables[1])]
+        st = ecco.new_stats(dev)
+        self.blocks = [ecco.encode(K, self.tables[0], stats=st), ecco.encode(V, self.tables[1], stats=st)]
+        self.stats, self.n_tensors = ecco.read_stats(st), 2
         self.new = [K.view(self.rows, self.S, self.D)[:, self.S - self.T:].contiguous(),
                     V.view(self.rows, self.S, self.D)[:, self.S - self.T:].contiguous()]
         self.out = [torch.empty((self.n, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
@@ -237,6 +315,7 @@ class KVWorkload(Workload):
 
 class C1Workload(Workload):
     name = "c1"
+    desc = "256 x 1024 bf16 matrix, N(0, 0.02^2) + 0.1% +-20 sigma outliers: encode + decode"
 
     def __init__(self, dev, seed_offset=0):
         import torch
@@ -244,10 +323,11 @@ class C1Workload(Workload):
         import entropy_coded_kv_b200 as ecco
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        self.desc = "256 x 1024 bf16 matrix, N(0, 0.02^2) + 0.1% +-20 sigma outliers: encode + decode"
         self.x = W.c1_matrix(device=dev, seed=0 + seed_offset)
         self.tables = ecco.Tables(learn_tables(W.c1_matrix(seed=0 + seed_offset)), dev)
-        self.blocks = ecco.encode(self.x, self.tables)
+        st = ecco.new_stats(dev)
+        self.blocks = ecco.encode(self.x, self.tables, stats=st)
+        self.stats = ecco.read_stats(st)
         self.out = torch.empty((2048, 128), dtype=torch.bfloat16, device=dev)
         self.launches_per_step = 2
         self.dec_ms = []
@@ -293,6 +373,8 @@ class C1Workload(Workload):
 
 class MLPWorkload(Workload):
     name = "mlp"
+    desc = ("14336 x 4096 bf16 weight, Student-t(5) x 0.02: encode, decode, fused decode+GEMV "
+            "at batch 1 and batch 16")
 
     def __init__(self, dev, seed_offset=0):
         import torch
@@ -300,13 +382,13 @@ class MLPWorkload(Workload):
         import entropy_coded_kv_b200 as ecco
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        self.desc = ("14336 x 4096 bf16 weight, Student-t(5) x 0.02: encode, decode, fused decode+GEMV "
-                     "at batch 1 and batch 16")
         self.w = W.c3_weight(device=dev, seed=3 + seed_offset)
         self.rows, self.cols = self.w.shape
         self.n = self.rows * self.cols // 128
         self.tables = ecco.Tables(learn_tables(self.w, seed=0), dev)
-        self.blocks = ecco.encode(self.w, self.tables)
+        st = ecco.new_stats(dev)
+        self.blocks = ecco.encode(self.w, self.tables, stats=st)
+        self.stats = ecco.read_stats(st)
         self.out = torch.empty((self.n, 128), dtype=torch.bfloat16, device=dev)
         self.x1 = W.activations(self.cols, 1, device=dev)
         self.x16 = W.activations(self.cols, 16, device=dev)
@@ -384,15 +466,16 @@ class ModelWorkload(Workload):
     """All 224 weight tensors of a 32-layer Llama-3-8B-shaped model: encode the
     whole set, decode the whole set (one multi-segment launch per 64 tensors)."""
     name = "model"
+    desc = ("Llama-3-8B-shaped weights, 32 layers x {q,k,v,o 4096/1024 x 4096; gate,up 14336 x 4096; "
+            "down 4096 x 14336}, Student-t(5) x 0.02, per-tensor tables: whole-model encode + decode")
 
     def __init__(self, dev, seed_offset=0):
         import torch
         import workloads as W
         import entropy_coded_kv_b200 as ecco
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        self.desc = ("Llama-3-8B-shaped weights, 32 layers x {q,k,v,o 4096/1024 x 4096; gate,up 14336 x 4096; "
-                     "down 4096 x 14336}, Student-t(5) x 0.02, per-tensor tables: whole-model encode + decode")
         self.w, self.tables = [], []
+        self.per_layer = len(W.C4_SHAPES)
         for layer in range(W.C4_LAYERS):
             for name, _, _ in W.C4_SHAPES:
                 t = W.c4_tensor(layer, name, device=dev, seed=4 + seed_offset)
@@ -403,7 +486,9 @@ class ModelWorkload(Workload):
         self.n = sum(t.numel() // 128 for t in self.w)
         self.enc = [ecco.Seg(tb, t, b) for tb, t, b in zip(self.tables, self.w, self.blocks)]
         self.dec = [ecco.Seg(tb, b, o.view(-1, 128)) for tb, b, o in zip(self.tables, self.blocks, self.out)]
-        ecco.encode_multi(self.enc)
+        st = ecco.new_stats(dev)
+        ecco.encode_multi(self.enc, st)
+        self.stats, self.n_tensors = ecco.read_stats(st), len(self.w)
         self.launches_per_step = 2 * ((len(self.w) + 63) // 64)
         self.ev = {"encode": [], "decode": []}
 
@@ -441,7 +526,26 @@ class ModelWorkload(Workload):
         return out
 
     def e2e_setup(self):
-        raise NotImplementedError("pinned host staging of the whole model (28 GB per step) is not run")
+        """Per layer: H2D of its 7 bf16 weights, encode_multi + decode_multi of
+        the layer, D2H of its blocks and decoded weights."""
+        torch, e = self.torch, self.ecco
+        self.h_w = [t.cpu().pin_memory() for t in self.w]
+        self.d_w = [torch.empty_like(t) for t in self.w]
+        k = self.per_layer
+        enc = [e.Seg(tb, dw, b) for tb, dw, b in zip(self.tables, self.d_w, self.blocks)]
+        layers = []
+        for i in range(0, len(self.w), k):
+            layers.append(([(self.h_w[j], self.d_w[j]) for j in range(i, i + k)],
+                           (lambda a, b: lambda: (e.encode_multi(a), e.decode_multi(b)))(enc[i:i + k],
+                                                                                      self.dec[i:i + k]),
+                           self.blocks[i:i + k] + self.out[i:i + k]))
+        self.stream = LayerStream(torch, self.dev, layers)
+        self.h2d, self.d2h = self.stream.h2d, self.stream.d2h
+        self.api = ("entropy_coded_kv_b200.encode_multi/decode_multi (C ABI), streamed per layer: H2D of the "
+                    "layer's bf16 weights from pinned host memory, D2H of its blocks and decoded weights")
+
+    def e2e_step(self):
+        self.stream.step()
 
     def cpu_sample(self, frac):
         import workloads as W
@@ -459,6 +563,9 @@ class LongCtxWorkload(Workload):
     """32 layers x K,V x [1, 8, 131072, 128] KV cache: decode the whole cache
     and append one token per layer (K and V), per step."""
     name = "longctx"
+    desc = ("long-context KV cache, 32 layers x K,V x [1, 8, 131072, 128] bf16 (17.2 GB), per-layer K/V "
+            "tables from [1, 8, 4096, 128] calibration samples: decode the whole cache + append one token "
+            "per layer (512 groups)")
     S = 131072
 
     def __init__(self, dev, seed_offset=0):
@@ -466,9 +573,6 @@ class LongCtxWorkload(Workload):
         import workloads as W
         import entropy_coded_kv_b200 as ecco
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        self.desc = ("long-context KV cache, 32 layers x K,V x [1, 8, 131072, 128] bf16 (17.2 GB), per-layer K/V "
-                     "tables from [1, 8, 4096, 128] calibration samples: decode the whole cache + append one token "
-                     "per layer (512 groups)")
         self.caches, self.tables = [], []
         for layer in range(32):
             K, V = W.c5_layer(layer, device=dev, seed=5 + seed_offset)
@@ -477,7 +581,9 @@ class LongCtxWorkload(Workload):
             self.tables += [ecco.Tables(ecco.learn_tables(c, seed=layer), dev) for c in (Kc, Vc)]  # GPU learner
             del Kc, Vc
         self.blocks = [torch.empty((c.numel() // 128, 64), dtype=torch.uint8, device=dev) for c in self.caches]
-        ecco.encode_multi([ecco.Seg(tb, c, b) for tb, c, b in zip(self.tables, self.caches, self.blocks)])
+        st = ecco.new_stats(dev)
+        ecco.encode_multi([ecco.Seg(tb, c, b) for tb, c, b in zip(self.tables, self.caches, self.blocks)], st)
+        self.stats, self.n_tensors = ecco.read_stats(st), len(self.caches)
         self.out = [torch.empty_like(c) for c in self.caches]
         self.new = [c.view(8, self.S, 128)[:, self.S - 1:].contiguous() for c in self.caches]
         app = ecco.kv_append_desc(8, 1, self.S, self.S - 1)
@@ -519,7 +625,30 @@ class LongCtxWorkload(Workload):
                 for k, evs in self.ev.items()}
 
     def e2e_setup(self):
-        raise NotImplementedError("pinned host staging of the whole cache (21.5 GB per step) is not run")
+        """Per layer: H2D of its compressed K and V caches and of the new
+        token, the append and the decode of the layer, D2H of the decoded K
+        and V."""
+        torch, e = self.torch, self.ecco
+        self.h_blocks = [b.cpu().pin_memory() for b in self.blocks]
+        self.h_new = [t.cpu().pin_memory() for t in self.new]
+        self.d_new = [torch.empty_like(t) for t in self.new]
+        app = e.kv_append_desc(8, 1, self.S, self.S - 1)
+        e2e_app = [e.Seg(tb, dn, b, app) for tb, dn, b in zip(self.tables, self.d_new, self.blocks)]
+        layers = []
+        for i in range(0, len(self.caches), 2):
+            ins = [(self.h_blocks[j], self.blocks[j]) for j in (i, i + 1)] + \
+                  [(self.h_new[j], self.d_new[j]) for j in (i, i + 1)]
+            layers.append((ins, (lambda a, b: lambda: (e.encode_multi(a), e.decode_multi(b)))(e2e_app[i:i + 2],
+                                                                                           self.dec[i:i + 2]),
+                           self.out[i:i + 2]))
+        self.stream = LayerStream(torch, self.dev, layers)
+        self.h2d, self.d2h = self.stream.h2d, self.stream.d2h
+        self.launches_e2e = 2 * len(layers)
+        self.api = ("entropy_coded_kv_b200.encode_multi/decode_multi (C ABI), streamed per layer: H2D of the "
+                    "layer's compressed K, V and new token from pinned host memory, D2H of its decoded K and V")
+
+    def e2e_step(self):
+        self.stream.step()
 
     def cpu_sample(self, frac):
         import workloads as W
@@ -541,25 +670,31 @@ class AttnWorkload(Workload):
     B, H, S, D, G = 8, 8, 4096, 128, 4
     path = "staged"  # or "fused": the single kernel that decodes inside the attention
 
+    @staticmethod
+    def describe(path):
+        how = ("staged decode+attention over all 4096 tokens (block decoder into a workspace scratch, then "
+               "the split kernel)" if path == "staged" else
+               "fused decode+attention over all 4096 tokens (one kernel decodes and attends)")
+        return ("decode-phase attention over a compressed Llama-3-8B-shaped layer KV cache: K, V "
+                "[8, 8, 4096, 128] as 64-byte blocks, 32 query heads (group 4); a step appends one "
+                "token's K and V (128 groups) and runs " + how)
+
     def __init__(self, dev, seed_offset=0):
         import torch
         import workloads as W
         import entropy_coded_kv_b200 as ecco
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        how = ("staged decode+attention over all 4096 tokens (block decoder into a workspace scratch, then "
-               "the split kernel)" if self.path == "staged" else
-               "fused decode+attention over all 4096 tokens (one kernel decodes and attends)")
-        self.desc = ("decode-phase attention over a compressed Llama-3-8B-shaped layer KV cache: K, V "
-                     "[8, 8, 4096, 128] as 64-byte blocks, 32 query heads (group 4); a step appends one "
-                     "token's K and V (128 groups) and runs " + how)
+        self.desc = self.describe(self.path)
         K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
         Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
         self.tables = [ecco.Tables(learn_tables(Kc, seed=0), dev), ecco.Tables(learn_tables(Vc, seed=0), dev)]
         self.rows = self.B * self.H
         self.n = self.rows * self.S
-        self.blocks = [ecco.encode(K, self.tables[0]).view(self.B, self.H, self.S, 64),
-                       ecco.encode(V, self.tables[1]).view(self.B, self.H, self.S, 64)]
+        st = ecco.new_stats(dev)
+        self.blocks = [ecco.encode(K, self.tables[0], stats=st).view(self.B, self.H, self.S, 64),
+                       ecco.encode(V, self.tables[1], stats=st).view(self.B, self.H, self.S, 64)]
+        self.stats, self.n_tensors = ecco.read_stats(st), 2
         self.new = [K.view(self.rows, self.S, self.D)[:, self.S - 1:].contiguous(),
                     V.view(self.rows, self.S, self.D)[:, self.S - 1:].contiguous()]
         self.append = ecco.kv_append_desc(self.rows, 1, self.S, self.S - 1)
@@ -649,6 +784,8 @@ class SelectWorkload(Workload):
     [8, 8, 4096, 128] layer with full-MSE pattern selection (64 patterns);
     setup also times and scores min/max and the 16-pattern variants."""
     name = "select"
+    desc = ("KV cache [8, 8, 4096, 128] K and V: encode with full-MSE pattern selection over 64 "
+            "patterns (524,288 groups); quality of min/max vs full-MSE selection, 64 and 16 patterns")
     B, H, S, D = 8, 8, 4096, 128
 
     def __init__(self, dev, seed_offset=0):
@@ -658,8 +795,6 @@ class SelectWorkload(Workload):
         from entropy_coded_kv_b200 import _lib
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev, self._lib = torch, ecco, dev, _lib
-        self.desc = ("KV cache [8, 8, 4096, 128] K and V: encode with full-MSE pattern selection over 64 "
-                     "patterns (524,288 groups); quality of min/max vs full-MSE selection, 64 and 16 patterns")
         K, V = W.c2_kv(device=dev, seed=1 + seed_offset)
         Kc, Vc = W.c2_calibration(device=dev, seed=2 + seed_offset)
         self.x = [K, V]
@@ -752,6 +887,8 @@ class ActWorkload(Workload):
     """Activation format: [8192, 4096] bf16 hidden states (Llama-3-8B width) in
     64-value groups; a step encodes and decodes all 524,288 groups."""
     name = "act"
+    desc = ("activations [8192, 4096] bf16 (channel-outlier hidden states) in the 2x format: "
+            "64-value groups, 524,288 blocks; encode + decode")
     T, D, GA = 8192, 4096, 64
 
     def __init__(self, dev, seed_offset=0):
@@ -760,13 +897,13 @@ class ActWorkload(Workload):
         import entropy_coded_kv_b200 as ecco
         from entropy_coded_kv_b200.calib import learn_tables
         self.torch, self.ecco, self.dev = torch, ecco, dev
-        self.desc = ("activations [8192, 4096] bf16 (channel-outlier hidden states) in the 2x format: "
-                     "64-value groups, 524,288 blocks; encode + decode")
         self.x = W.hidden_states(self.T, self.D, seed=6 + seed_offset, device=dev)
         self.tables = ecco.Tables(learn_tables(W.hidden_states(2048, self.D, seed=61 + seed_offset),
                                                seed=0, group=self.GA), dev)
         self.n = self.x.numel() // self.GA
-        self.blocks = ecco.encode_act(self.x, self.tables)
+        st = ecco.new_stats(dev)
+        self.blocks = ecco.encode_act(self.x, self.tables, stats=st)
+        self.stats, self.group = ecco.read_stats(st), self.GA
         self.out = torch.empty((self.n, self.GA), dtype=torch.bfloat16, device=dev)
         self.launches_per_step = 2
         self.dec_ms = []
@@ -820,6 +957,106 @@ class ActWorkload(Workload):
 
 WORKLOADS = {"act": ActWorkload, "kv": KVWorkload, "c1": C1Workload, "mlp": MLPWorkload, "model": ModelWorkload,
              "longctx": LongCtxWorkload, "attn": AttnWorkload, "select": SelectWorkload}
+
+
+# ------------------------------------------------------------------ host-only samples (reference arm)
+def host_sample(name):
+    """A bounded sample of workload `name` built on the host alone, for the
+    oracle arm: inputs from `workloads` on the CPU (the workload's
+    distribution and seeds, at a reduced size where the full one would take
+    minutes to generate or run), tables from the host learner
+    (entropy_coded_kv_b200.calib, numpy) on a small calibration sample, blocks
+    from the oracle's own encoder.  No device and no libecco_b200.so."""
+    import numpy as np
+    import torch
+    import oracle
+    import workloads as W
+    from entropy_coded_kv_b200.calib import learn_tables
+
+    def bits(t):
+        return W.bf16_bits(t)
+
+    def enc(blob, xb, gs=128):
+        return oracle.encode(blob, xb, nthreads=os.cpu_count() or 1, gs=gs)[0]
+
+    if name == "c1":
+        x = W.c1_matrix(seed=0)
+        blob = learn_tables(x)
+        xb = bits(x)
+        return {"enc": [(blob, xb)], "dec": [(blob, enc(blob, xb))], "bytes": 2 * 2048 * 256,
+                "what": "the whole step (encode 2048 groups + decode 2048 blocks)"}
+    if name in ("kv", "select"):
+        K, V = W.c2_kv(seed=1)
+        cal = W.kv_cache((1, 8, 256, 128), 2)
+        blobs = [learn_tables(cal[0], seed=0), learn_tables(cal[1], seed=0)]
+        if name == "select":
+            k = 2048
+            xs = [bits(t.reshape(-1, 128)[:k]) for t in (K, V)]
+            return {"enc": list(zip(blobs, xs)), "dec": [], "select": 1, "bytes": 2 * k * 256,
+                    "what": f"full-MSE encode of {2 * k} groups (1/{524288 // k} of a step)"}
+        new = [bits(t.reshape(64, 4096, 128)[:, 4032:]) for t in (K, V)]
+        dec = [(b, enc(b, bits(t))) for b, t in zip(blobs, (K, V))]
+        return {"enc": list(zip(blobs, new)), "dec": dec, "bytes": 2 * 524288 * 256 + 2 * 8192 * 256,
+                "what": "the whole step (encode 8,192 groups of K and of V + decode 524,288 blocks of each)"}
+    if name == "mlp":
+        g = W._gen(3, "cpu")
+        w = (W.student_t((896, 4096), 5, g, "cpu") * 0.02).to(dtype=torch.bfloat16)
+        blob = learn_tables(w[:64])
+        xb = bits(w)
+        n = xb.size // 128
+        return {"enc": [(blob, xb)], "dec": [(blob, enc(blob, xb))], "bytes": 2 * n * 256,
+                "what": f"encode + decode of {n} groups (896 of 14,336 rows; GEMV not sampled)"}
+    if name == "model":
+        encs, decs, nb = [], [], 0
+        shape_blob = {}
+        for layer in range(W.C4_LAYERS):
+            for i, (sh, rows, cols) in enumerate(W.C4_SHAPES):
+                g = W._gen(4 * 1000 + layer * len(W.C4_SHAPES) + i, "cpu")
+                k = max(8, rows * cols // 128 // 1000)
+                t = (W.student_t((k, 128), 5, g, "cpu") * 0.02).to(dtype=torch.bfloat16)
+                if sh not in shape_blob:
+                    cal = (W.student_t((2048, 128), 5, W._gen(40 + i, "cpu"), "cpu") * 0.02).to(dtype=torch.bfloat16)
+                    shape_blob[sh] = learn_tables(cal)
+                blob, xb = shape_blob[sh], bits(t)
+                encs.append((blob, xb))
+                decs.append((blob, enc(blob, xb)))
+                nb += k
+        return {"enc": encs, "dec": decs, "bytes": 2 * nb * 256,
+                "what": f"encode + decode of {nb} groups across all 224 tensors (1/1000 of each; one table set "
+                        f"per tensor shape)"}
+    if name == "longctx":
+        encs, decs, nb = [], [], 0
+        tok = 1311  # ~1% of the 131,072 tokens of every head
+        for layer in range(32):
+            kv = W.kv_cache((1, 8, tok, 128), 5 * 1000 + layer)
+            cal = W.kv_cache((1, 8, 256, 128), 105 * 1000 + layer)
+            for t, c in zip(kv, cal):
+                blob = learn_tables(c, seed=layer)
+                xb = bits(t).reshape(8, tok, 128)
+                encs.append((blob, np.ascontiguousarray(xb[:, -1])))
+                decs.append((blob, enc(blob, xb.reshape(-1, 128))))
+                nb += 8 * tok
+        return {"enc": encs, "dec": decs, "bytes": nb * 256 + 512 * 256,
+                "what": f"the per-step append (512 groups) + decode of {nb} blocks ({tok} of 131,072 tokens of "
+                        f"every head of all 64 caches)"}
+    if name == "attn":
+        K, V = W.kv_cache((1, 1, 4096, 128), 1)
+        cal = W.kv_cache((1, 8, 256, 128), 2)
+        blobs = [learn_tables(cal[0], seed=0), learn_tables(cal[1], seed=0)]
+        kb = [enc(b, bits(t)).reshape(1, 4096, 64) for b, t in zip(blobs, (K, V))]
+        q = torch.randn(1, 4, 128, generator=W._gen(77, "cpu")).to(torch.bfloat16)
+        xs = [bits(t.reshape(4096, 128)[-1:]) for t in (K, V)]
+        return {"enc": list(zip(blobs, xs)), "dec": [], "attn": (blobs, kb, bits(q), 4096, 128 ** -0.5),
+                "bytes": 2 * 4096 * 256 + 2 * 256,
+                "what": "append + attention for 1 of 64 (batch, KV head) pairs (8,192 blocks decoded)"}
+    if name == "act":
+        x = W.hidden_states(128, 4096, seed=6)
+        blob = learn_tables(W.hidden_states(32, 4096, seed=61), seed=0, group=64)
+        xb = bits(x)
+        n = xb.size // 64
+        return {"enc": [(blob, xb)], "dec": [(blob, enc(blob, xb, 64))], "gs": 64, "bytes": 2 * n * 128,
+                "what": f"encode + decode of {n} activation groups (128 of 8,192 tokens)"}
+    raise KeyError(name)
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -974,6 +1211,9 @@ def main():
     }
     if ops:
         line["ops"] = ops
+    summary = wl.stats_summary()
+    if summary:
+        line["stats"] = summary
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1020,16 +1260,12 @@ def traffic_for(workload, kernel):
 
 def run_reference(args, world):
     """The CPU oracle as the reference arm: each step is a bounded sample of the
-    workload, timed with the wall clock on the host cores."""
-    import torch
-    dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
-    if dev is None:
-        print(json.dumps({"impl": "reference", "unavailable": "workload inputs are generated on a CUDA device"}))
-        return
-    AttnWorkload.path = args.attention
-    wl = WORKLOADS[args.workload](dev)
+    workload (host_sample: built without a device or the product library),
+    timed with the wall clock on the host cores."""
+    cls = WORKLOADS[args.workload]
+    desc = AttnWorkload.describe(args.attention) if cls is AttnWorkload else cls.desc
     cores = os.cpu_count() or 1
-    sample = wl.cpu_sample(wl.cpu_frac())
+    sample = host_sample(args.workload)
     for _ in range(max(1, min(args.warmup, 2))):
         time_oracle(sample, cores)
     t0 = time.perf_counter()
@@ -1041,12 +1277,11 @@ def run_reference(args, world):
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.desc, "sample": sample["what"]},
+        "config": {"workload": desc, "sample": sample["what"]},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": sample["what"]},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
-
 
 if __name__ == "__main__":
     main()

@@ -7,19 +7,19 @@
 
 namespace ecco {
 
+// SM count of the current device, looked up once per device (safe from
+// several host threads: each slot is written with the same value).
 int device_sm_count()
 {
-    static int cached_dev = -1;
-    static int cached_sms = 0;
+    static std::atomic<int> cached[kMaxDeviceBits];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev != cached_dev) {
-        int sms = 0;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cached_sms = sms > 0 ? sms : 1;
-        cached_dev = dev;
-    }
-    return cached_sms;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    const bool slot = dev >= 0 && dev < kMaxDeviceBits;
+    int sms = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
+    if (sms > 0) return sms;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 1;
+    if (slot) cached[dev].store(sms, std::memory_order_relaxed);
+    return sms;
 }
 
 namespace {
@@ -177,10 +177,12 @@ extern "C" size_t ecco_decode_attention_workspace_bytes(int batch, int kv_heads,
            (size_t)attention_splits(seq_len);
 }
 
-extern "C" int ecco_decode_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
-                                     const uint8_t* vblk, int64_t s_cap, int batch, int kv_heads,
-                                     int group, int seq_len, const uint16_t* q, float scale, float* out,
-                                     void* ws, size_t ws_bytes, void* stream)
+namespace ecco {
+// Checks shared by the attention entry points, in the order the header states:
+// tables, sizes, pointers, then alignment of the inputs and the output.
+int check_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk, const uint8_t* vblk,
+                    int64_t s_cap, int batch, int kv_heads, int group, int seq_len, const uint16_t* q,
+                    const float* out)
 {
     int rc = check_tables(kt);
     if (rc) return rc;
@@ -188,11 +190,24 @@ extern "C" int ecco_decode_attention(const ecco_tables* kt, const ecco_tables* v
     if (batch < 1 || kv_heads < 1 || group < 1 || group > 8 || seq_len < 1 || s_cap < seq_len)
         return ECCO_ERR_ARG;
     if ((int64_t)batch * kv_heads > 65535 || s_cap > ((int64_t)1 << 34)) return ECCO_ERR_ARG;
-    if (!kblk || !vblk || !q || !out || !ws) return ECCO_ERR_ARG;
-    if (ws_bytes < ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len)) return ECCO_ERR_ARG;
+    if (!kblk || !vblk || !q || !out) return ECCO_ERR_ARG;
     if (!aligned16(kblk) || !aligned16(vblk) || (reinterpret_cast<uintptr_t>(q) & 1u) ||
-        (reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 3u))
+        (reinterpret_cast<uintptr_t>(out) & 3u))
         return ECCO_ERR_ALIGN;
+    return ECCO_OK;
+}
+}  // namespace ecco
+
+extern "C" int ecco_decode_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
+                                     const uint8_t* vblk, int64_t s_cap, int batch, int kv_heads,
+                                     int group, int seq_len, const uint16_t* q, float scale, float* out,
+                                     void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, out);
+    if (rc) return rc;
+    if (!ws) return ECCO_ERR_ARG;
+    if (ws_bytes < ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len)) return ECCO_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(ws) & 3u) return ECCO_ERR_ALIGN;
     return status(launch_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, scale,
                                    out, static_cast<float*>(ws), (cudaStream_t)stream));
 }
@@ -219,18 +234,12 @@ extern "C" int ecco_decode_attention_staged(const ecco_tables* kt, const ecco_ta
                                             int group, int seq_len, const uint16_t* q, float scale, float* out,
                                             void* ws, size_t ws_bytes, void* stream)
 {
-    int rc = check_tables(kt);
+    int rc = check_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, out);
     if (rc) return rc;
-    if ((rc = check_tables(vt))) return rc;
-    if (batch < 1 || kv_heads < 1 || group < 1 || group > 8 || seq_len < 1 || s_cap < seq_len)
-        return ECCO_ERR_ARG;
-    if ((int64_t)batch * kv_heads > 65535 || s_cap > ((int64_t)1 << 34)) return ECCO_ERR_ARG;
-    if (!kblk || !vblk || !q || !out || !ws) return ECCO_ERR_ARG;
+    if (!ws) return ECCO_ERR_ARG;
     if (ws_bytes < ecco_decode_attention_staged_workspace_bytes(batch, kv_heads, group, seq_len))
         return ECCO_ERR_ARG;
-    if (!aligned16(kblk) || !aligned16(vblk) || (reinterpret_cast<uintptr_t>(q) & 1u) ||
-        (reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 3u))
-        return ECCO_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(ws) & 3u) return ECCO_ERR_ALIGN;
     // partials first, then the decoded-row scratch from the next 256-byte boundary
     const uintptr_t sc = (reinterpret_cast<uintptr_t>(ws) + staged_partials_bytes(batch, kv_heads, group, seq_len) +
                           kScratchAlign - 1) / kScratchAlign * kScratchAlign;

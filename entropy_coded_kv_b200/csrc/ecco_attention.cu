@@ -497,16 +497,9 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict
 template <int G, bool STAGED>
 cudaError_t configure_attn()
 {
-    static int configured = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured != dev) {
-        cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<G, STAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(STAGED ? kAttnSmemStaged : kAttnSmem));
-        if (e != cudaSuccess) return e;
-        configured = dev;
-    }
-    return cudaSuccess;
+    static std::atomic<uint64_t> configured{0};
+    return set_max_smem_once(configured, (const void*)attn_split_kernel<G, STAGED>,
+                             STAGED ? kAttnSmemStaged : kAttnSmem);
 }
 
 template <int G>
@@ -622,12 +615,12 @@ extern "C" int ecco_decode_attention_static(const ecco_tables* kt, const ecco_ta
                                             int group, int seq_len, const uint16_t* q, float scale, float* out,
                                             void* stream)
 {
+    // the same checks, in the same order, as ecco_decode_attention; then the size limit
+    int rc = ecco::check_attention(kt, vt, kblk, vblk, s_cap, batch, kv_heads, group, seq_len, q, out);
+    if (rc) return rc;
     const size_t need = ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len);
-    if (need == 0 || !kt || !vt) return ECCO_ERR_ARG;
     if (need > (size_t)ECCO_ATTENTION_STATIC_WS_BYTES) return ECCO_ERR_WORKSPACE;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return ECCO_ERR_CUDA;
-    if (dev != kt->device || dev != vt->device) return ECCO_ERR_DEVICE;
+    const int dev = kt->device;  // the current device (checked above)
     if (dev < 0 || dev >= kMaxDevices) return ECCO_ERR_UNSUPPORTED;
     void* ws = g_static_ws_addr[dev].load(std::memory_order_acquire);
     if (!ws) {

@@ -196,15 +196,9 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
 template <bool WIDE, int MAXSEG, int G = kG>
 cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
 {
-    static int configured = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured != dev) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<WIDE, MAXSEG, G>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dec_smem<G>());
-        if (e != cudaSuccess) return e;
-        configured = dev;
-    }
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = set_max_smem_once(configured, (const void*)decode_kernel<WIDE, MAXSEG, G>, dec_smem<G>());
+    if (e != cudaSuccess) return e;
     int64_t want = (P.total + dec_threads<G>() - 1) / dec_threads<G>();
     int64_t cap = device_sm_count();
     int grid = (int)(want < cap ? want : cap);

@@ -294,13 +294,9 @@ size_t gemm_tc_smem() { return kTcSmem; }
 cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                            const uint16_t* x, int batch, float* y, cudaStream_t s)
 {
-    static int configured = -1;
-    if (configured != t->device) {
-        cudaError_t e =
-            cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
-        if (e != cudaSuccess) return e;
-        configured = t->device;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (cudaError_t e0 = set_max_smem_once(configured, (const void*)gemm_tc_kernel, kTcSmem); e0 != cudaSuccess)
+        return e0;
     cudaError_t e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)batch * (size_t)rows, s);
     if (e != cudaSuccess) return e;
     const int64_t gpr = cols / kG;

@@ -179,13 +179,9 @@ template <int B>
 cudaError_t run_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                      const uint16_t* x, int batch, float* y, cudaStream_t s)
 {
-    static int configured_dev = -1;
-    if (configured_dev != t->device) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)gv_smem<B>());
-        if (e != cudaSuccess) return e;
-        configured_dev = t->device;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (cudaError_t e0 = set_max_smem_once(configured, (const void*)gemv_kernel<B>, gv_smem<B>()); e0 != cudaSuccess)
+        return e0;
     cudaError_t e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)batch * (size_t)rows, s);
     if (e != cudaSuccess) return e;
     const int64_t gpr = cols / kG;

@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/ecco.h"
 
 namespace ecco {
@@ -103,6 +105,32 @@ cudaError_t learn_tables(const uint16_t* x, int64_t n_groups, int G, int npat, u
 int huffman_lengths(const double* w, int n, int max_len, uint8_t* lens);
 
 int device_sm_count();
+
+// Argument checks of the attention entry points (tables, sizes, pointers,
+// alignment of blocks, q and out); ECCO_OK or the error code to return.
+int check_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk, const uint8_t* vblk,
+                    int64_t s_cap, int batch, int kv_heads, int group, int seq_len, const uint16_t* q,
+                    const float* out);
+
+// Devices a per-kernel "already configured" bit set can name; a device index
+// at or beyond it is configured on every launch (correct, just slower).
+constexpr int kMaxDeviceBits = 64;
+
+// Raises `fn`'s dynamic shared-memory limit to `bytes` on the current device,
+// once per device: `done` holds one bit per device whose call succeeded.
+// Safe to call from several host threads at once (a race only repeats the
+// idempotent attribute call).
+inline cudaError_t set_max_smem_once(std::atomic<uint64_t>& done, const void* fn, size_t bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < kMaxDeviceBits) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // ------------------------------------------------------------ device helpers
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }

@@ -550,10 +550,9 @@ cudaError_t learn_tables(const uint16_t* x, int64_t n_groups, int G, int npat, u
         (e = d_hist.alloc(sizeof(int) * (size_t)n * kNSym)))
         return e;
     {
-        cudaError_t ea = cudaFuncSetAttribute(refine_kernel<kG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              (int)kRefineSmem);
-        cudaError_t eb = cudaFuncSetAttribute(refine_kernel<kGAct>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              (int)kRefineSmem);
+        static std::atomic<uint64_t> done_g{0}, done_a{0};
+        cudaError_t ea = set_max_smem_once(done_g, (const void*)refine_kernel<kG>, kRefineSmem);
+        cudaError_t eb = set_max_smem_once(done_a, (const void*)refine_kernel<kGAct>, kRefineSmem);
         if (ea != cudaSuccess) return ea;
         if (eb != cudaSuccess) return eb;
     }

@@ -247,9 +247,11 @@ int ecco_decode_attention_staged(const ecco_tables* k_tables, const ecco_tables*
  * callers that cannot allocate device memory where they run attention: a
  * plain-C host loop has no caching allocator to draw a workspace from, and
  * cudaMalloc can synchronize the device and fail under memory pressure.
- *   - Requests whose workspace (ecco_decode_attention_workspace_bytes) exceeds
- *     ECCO_ATTENTION_STATIC_WS_BYTES return ECCO_ERR_WORKSPACE and enqueue
- *     nothing; other arguments and errors are those of ecco_decode_attention.
+ *   - The arguments are checked first, in ecco_decode_attention's order and
+ *     with its error codes (tables, sizes, pointers, alignment).  A valid
+ *     request whose workspace (ecco_decode_attention_workspace_bytes) exceeds
+ *     ECCO_ATTENTION_STATIC_WS_BYTES then returns ECCO_ERR_WORKSPACE; either
+ *     way nothing is enqueued.
  *   - Nothing in the workspace needs to start at zero: every split writes all
  *     of its partial results before the merge reads them.
  *   - The first call on each device looks up the workspace's address with that

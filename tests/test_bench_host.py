@@ -1,6 +1,6 @@
 """Host-side logic of bench.py (no GPU): the committed DRAM-traffic entries and
-their source hashes, the peak lookup, and the reference arm's line on a
-machine without a CUDA device."""
+their source hashes, the peak lookup, and the reference arm (the oracle alone,
+on host-built samples)."""
 from __future__ import annotations
 
 import json
@@ -59,10 +59,28 @@ def test_attention_workload_defaults_to_the_staged_path():
     assert bench.AttnWorkload.path == "staged"
 
 
-@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device line")
-def test_reference_arm_without_a_device_prints_its_unavailable_line():
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference"],
-                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+_RUN_AND_LIST_LIBS = (
+    "import runpy, sys; sys.argv = ['bench.py'] + sys.argv[1:]; "
+    "runpy.run_path('bench.py', run_name='__main__'); "
+    "maps = open('/proc/self/maps').read(); "
+    "print('LIBS', int('libecco_b200' in maps), int('libecco_oracle' in maps))")
+
+
+@pytest.mark.parametrize("workload", [None, "c1", "attn"])
+def test_reference_arm_runs_the_oracle_alone(workload):
+    """The reference arm times the oracle on a host-built sample: it needs no
+    device and never maps the product library."""
+    args = ["--impl", "reference", "--steps", "1", "--warmup", "1"]
+    if workload:
+        args += ["--workload", workload]
+    r = subprocess.run([sys.executable, "-c", _RUN_AND_LIST_LIBS] + args, capture_output=True, text=True,
+                       timeout=600, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
-    line = json.loads(r.stdout.strip().splitlines()[-1])
-    assert line["impl"] == "reference" and "unavailable" in line
+    out = r.stdout.strip().splitlines()
+    line = json.loads(out[-2])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    want = bench.WORKLOADS[workload or "longctx"]
+    if want is not bench.AttnWorkload:
+        assert line["config"]["workload"] == want.desc
+    assert out[-1] == "LIBS 0 1"

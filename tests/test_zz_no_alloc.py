@@ -39,14 +39,27 @@ def _close(a, b):
     np.testing.assert_allclose(a, b, rtol=1e-5, atol=1e-6 * float(np.abs(b).max()))
 
 
+def _device_allocations():
+    """(caching-allocator allocations so far, bytes free on the device)."""
+    torch.cuda.synchronize()
+    return torch.cuda.memory_stats(DEV).get("allocation.all.allocated", 0), torch.cuda.mem_get_info(DEV)[0]
+
+
 @pytest.mark.parametrize("B,H,G,S_cap,n", [(2, 2, 4, 1300, 1237), (1, 3, 8, 700, 513), (8, 8, 4, 4096, 4096)])
 def test_static_workspace_matches_caller_workspace(B, H, G, S_cap, n):
     tk, tv, kb, vb, q = _case(B, H, G, S_cap, seed=n)
     want = ecco.decode_attention(kb, vb, tk, tv, q, n, 0.0884)
     out = torch.empty_like(want)
-    for _ in range(2):
+    for i in range(2):
         out.fill_(float("nan"))
+        before = _device_allocations()
         ecco.decode_attention_static(kb, vb, tk, tv, q, n, 0.0884, out=out)
+        # the call itself allocates nothing: no caching-allocator block and,
+        # after the first call's one-time set-up, no device memory at all
+        after = _device_allocations()
+        assert after[0] == before[0]
+        if i == 1:
+            assert after[1] == before[1]
         _close(out, want)
 
 
@@ -65,5 +78,17 @@ def test_largest_request_that_fits_and_first_that_does_not():
         ctypes.c_void_p(q.data_ptr()), 0.0884, ctypes.c_void_p(out.data_ptr()), None)
     assert rc == _lib.ECCO_ERR_WORKSPACE
     assert "static" in _lib.strerror(rc)
+    # argument errors come first, as in ecco_decode_attention: an oversized
+    # request with a null table handle or a misaligned q is an argument error
+    L = _lib.load()
+    rc = L.ecco_decode_attention_static(None, tv.handle, ctypes.c_void_p(kb.data_ptr()), ctypes.c_void_p(vb.data_ptr()),
+                                        over, 1, 1, 8, over, ctypes.c_void_p(q.data_ptr()), 0.0884,
+                                        ctypes.c_void_p(out.data_ptr()), None)
+    assert rc == _lib.ECCO_ERR_ARG
+    rc = L.ecco_decode_attention_static(tk.handle, tv.handle, ctypes.c_void_p(kb.data_ptr()),
+                                        ctypes.c_void_p(vb.data_ptr()), over, 1, 1, 8, over,
+                                        ctypes.c_void_p(q.data_ptr() + 1), 0.0884, ctypes.c_void_p(out.data_ptr()),
+                                        None)
+    assert rc == _lib.ECCO_ERR_ALIGN
     torch.cuda.synchronize()
     assert torch.count_nonzero(out) == 0  # nothing was enqueued
