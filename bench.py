@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="model / longctx: layers built (32 = the full configuration; fewer for profiling captures)")
     return ap.parse_args()
 
 
@@ -466,6 +468,7 @@ class ModelWorkload(Workload):
     """All 224 weight tensors of a 32-layer Llama-3-8B-shaped model: encode the
     whole set, decode the whole set (one multi-segment launch per 64 tensors)."""
     name = "model"
+    layers = 32  # bench.py --layers: fewer only for profiling captures
     desc = ("Llama-3-8B-shaped weights, 32 layers x {q,k,v,o 4096/1024 x 4096; gate,up 14336 x 4096; "
             "down 4096 x 14336}, Student-t(5) x 0.02, per-tensor tables: whole-model encode + decode")
 
@@ -476,7 +479,8 @@ class ModelWorkload(Workload):
         self.torch, self.ecco, self.dev = torch, ecco, dev
         self.w, self.tables = [], []
         self.per_layer = len(W.C4_SHAPES)
-        for layer in range(W.C4_LAYERS):
+        self.layers = min(self.layers, W.C4_LAYERS)
+        for layer in range(self.layers):
             for name, _, _ in W.C4_SHAPES:
                 t = W.c4_tensor(layer, name, device=dev, seed=4 + seed_offset)
                 self.w.append(t)
@@ -563,6 +567,7 @@ class LongCtxWorkload(Workload):
     """32 layers x K,V x [1, 8, 131072, 128] KV cache: decode the whole cache
     and append one token per layer (K and V), per step."""
     name = "longctx"
+    layers = 32  # bench.py --layers: fewer only for profiling captures
     desc = ("long-context KV cache, 32 layers x K,V x [1, 8, 131072, 128] bf16 (17.2 GB), per-layer K/V "
             "tables from [1, 8, 4096, 128] calibration samples: decode the whole cache + append one token "
             "per layer (512 groups)")
@@ -574,7 +579,7 @@ class LongCtxWorkload(Workload):
         import entropy_coded_kv_b200 as ecco
         self.torch, self.ecco, self.dev = torch, ecco, dev
         self.caches, self.tables = [], []
-        for layer in range(32):
+        for layer in range(min(self.layers, 32)):
             K, V = W.c5_layer(layer, device=dev, seed=5 + seed_offset)
             Kc, Vc = W.c5_calibration(layer, device=dev, seed=105 + seed_offset)
             self.caches += [K, V]
@@ -1124,7 +1129,10 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     AttnWorkload.path = args.attention
+    ModelWorkload.layers = LongCtxWorkload.layers = args.layers
     wl = WORKLOADS[args.workload](dev, seed_offset=0)
+    if getattr(wl, "layers", 32) != 32:
+        wl.desc = f"{wl.desc} [only {wl.layers} of 32 layers built]"
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
     for _ in range(max(3, args.warmup)):

@@ -16,6 +16,7 @@ ECCO_ERR_CUDA = -4
 ECCO_ERR_DEVICE = -5
 ECCO_ERR_UNSUPPORTED = -6
 ECCO_ERR_WORKSPACE = -7
+ECCO_ERR_TIMEOUT = -8
 ATTENTION_STATIC_WS_BYTES = 4 << 20
 SELECT_MINMAX = 0
 SELECT_MSE = 1
@@ -29,6 +30,7 @@ EXPORTED = [
     "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static", "ecco_select_encode_ex",
     "ecco_select_encode_act", "ecco_decode_act", "ecco_learn_tables", "ecco_huffman_lengths",
     "ecco_decode_attention_staged", "ecco_decode_attention_staged_workspace_bytes",
+    "ecco_selftest_wait_timeout",
 ]
 
 
@@ -79,6 +81,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_strerror.restype = ctypes.c_char_p
     L.ecco_abi_version.argtypes = []
     L.ecco_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    L.ecco_selftest_wait_timeout.argtypes = [P]
     L.ecco_decode_attention_workspace_bytes.argtypes = [I, I, I, I]
     L.ecco_decode_attention_static.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P]
     L.ecco_decode_attention.argtypes = [P, P, P, P, I64, I, I, I, I, P, ctypes.c_float, P, P,

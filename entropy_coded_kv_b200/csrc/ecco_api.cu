@@ -138,6 +138,7 @@ extern "C" int ecco_decode_gemv(const ecco_tables* t, const uint8_t* blocks, int
                                                  (cudaStream_t)stream));
     if (!blocks || !x) return ECCO_ERR_ARG;
     if (!aligned16(blocks) || !aligned16(x) || !aligned16(y)) return ECCO_ERR_ALIGN;
+    if (batch > 4 && timeout_raised()) return ECCO_ERR_TIMEOUT;  // an earlier tensor-core launch gave up
     return status(launch_gemv(t, blocks, rows, cols, x, batch, y, (cudaStream_t)stream));
 }
 
@@ -285,9 +286,15 @@ extern "C" const char* ecco_strerror(int code)
         case ECCO_ERR_DEVICE: return "current device is not the tables' device";
         case ECCO_ERR_UNSUPPORTED: return "device is not sm_100";
         case ECCO_ERR_WORKSPACE: return "request needs more than the static attention workspace";
+        case ECCO_ERR_TIMEOUT: return "a bounded device wait gave up in an earlier tensor-core launch";
         default: return "unknown error";
     }
 }
 
 extern "C" int ecco_abi_version(void) { return 1; }
 
+extern "C" int ecco_selftest_wait_timeout(void* stream)
+{
+    if (!timeout_flag()) return ECCO_ERR_CUDA;
+    return status(launch_wait_timeout_selftest((cudaStream_t)stream));
+}

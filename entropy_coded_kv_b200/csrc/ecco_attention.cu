@@ -172,13 +172,13 @@ __device__ __forceinline__ void for_records(const Stream& st, const uint32_t* ws
 // Decodes the 32 symbols of quarter `qd` of this thread's block into its row
 // of the warp's staging tile; the symbols (nibbles) go to the thread's column
 // nb[k * kAtStride], k = chunk, for the record pass.
-__device__ __forceinline__ void decode_quarter(Stream& st, const uint8_t* lut, const uint32_t* ws,
+__device__ __forceinline__ void decode_quarter(Stream& st, uint32_t lkey, const uint32_t* ws,
                                                const ValuePlanes& vp, uint32_t* row, uint32_t* nb, int qd)
 {
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t w[4];
-        nb[(qd * 4 + c4) * kAtStride] = chunk_values(st, lut, ws, kAtStride, vp, w);
+        nb[(qd * 4 + c4) * kAtStride] = chunk_values(st, lkey, ws, kAtStride, vp, w);
         *reinterpret_cast<uint4*>(row + 4 * c4) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
@@ -342,13 +342,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         const float s = load_block(A.kblk + blk * ECCO_BLOCK_BYTES, have, q0, q1, q2, q3, A.ktb->S_t);
         stage_words(ws, kAtStride, q0, q1, q2, q3);
         const ValuePlanes vp = make_planes(s, s_Ct, (int)((q0.x >> 8) & 63u));
-        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
+        const uint32_t lkey = lut_key(s_lut, (q0.x >> 8) & 255u);
         Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
         // qrow[j] = q[gid][2 (tig + j)], q[gid][2 (tig + j) + 1]
         const uint32_t* qrow = reinterpret_cast<const uint32_t*>(s_qb + gid * kQbRow) + tig;
 #pragma unroll
         for (int qd = 0; qd < 4; ++qd) {
-            decode_quarter(st, lut, ws, vp, row, nb, qd);
+            decode_quarter(st, lkey, ws, vp, row, nb, qd);
             __syncwarp();
             k_quarter_mma(S, qrow, stage_sh, lane, qd);
             __syncwarp();
@@ -448,11 +448,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         const float s = load_block(A.vblk + blk * ECCO_BLOCK_BYTES, have, q0, q1, q2, q3, A.vtb->S_t);
         stage_words(ws, kAtStride, q0, q1, q2, q3);
         const ValuePlanes vp = make_planes(s, s_Ct, (int)((q0.x >> 8) & 63u));
-        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
+        const uint32_t lkey = lut_key(s_lut, (q0.x >> 8) & 255u);
         Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 #pragma unroll
         for (int qd = 0; qd < 4; ++qd) {
-            decode_quarter(st, lut, ws, vp, row, nb, qd);
+            decode_quarter(st, lkey, ws, vp, row, nb, qd);
             __syncwarp();
             v_quarter_mma<G>(s_acc, pa, stage_sh, lane, gid, tig, qd);
             __syncwarp();

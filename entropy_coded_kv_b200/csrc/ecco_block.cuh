@@ -32,14 +32,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Ct: centroids transposed, Ct[j * 64 + p], row 15 = 1.0 (the scale element).
+// Ct: centroids transposed, Ct[j * 64 + p], row 15 = 1.0 (the scale element);
+// in shared memory, or read through the read-only cache when GLOBAL.
+template <bool GLOBAL = false>
 __device__ __forceinline__ ValuePlanes make_planes(float s, const float* Ct, int p)
 {
     ValuePlanes v;
+    auto c = [&](int j) { return GLOBAL ? __ldg(Ct + j * kNPat + p) : Ct[j * kNPat + p]; };
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        uint32_t a = pack_bf16x2(__fmul_rn(s, Ct[(4 * q + 0) * kNPat + p]), __fmul_rn(s, Ct[(4 * q + 1) * kNPat + p]));
-        uint32_t b = pack_bf16x2(__fmul_rn(s, Ct[(4 * q + 2) * kNPat + p]), __fmul_rn(s, Ct[(4 * q + 3) * kNPat + p]));
+        uint32_t a = pack_bf16x2(__fmul_rn(s, c(4 * q + 0)), __fmul_rn(s, c(4 * q + 1)));
+        uint32_t b = pack_bf16x2(__fmul_rn(s, c(4 * q + 2)), __fmul_rn(s, c(4 * q + 3)));
         v.lo[q] = __byte_perm(a, b, 0x6420);
         v.hi[q] = __byte_perm(a, b, 0x7531);
     }
@@ -88,19 +91,30 @@ __device__ __forceinline__ void refill(Stream& st, const uint32_t* ws, int strid
     }
 }
 
+// Shared-memory key of a block's decode table: the table's address (tables
+// start on a 256-byte boundary of the shared window, see aligned_smem) OR-ed
+// with its swizzle.  `hdr` = header bits 8..15 = codebook * 64 + pattern, the
+// table index.  Entry e of table t sits at byte e ^ ((t & 31) << 2): its
+// 4-byte word is XOR-ed with the low 5 bits of t, so lanes that read the same
+// entry of different tables -- common, since canonical codes give the short,
+// frequent codewords the same low stream bits in every codebook -- land in
+// different banks.  (ecco_tables.cu builds the tables in this layout.)
+__device__ __forceinline__ uint32_t lut_key(const uint8_t* s_lut, uint32_t hdr)
+{
+    return ((uint32_t)__cvta_generic_to_shared(s_lut) + hdr * 256u) | ((hdr & 31u) << 2);
+}
+
 // Decodes 8 symbols.  Returns their nibbles (symbol k in bits 4k..4k+3); `kv`
 // = number of them that end
 // at or before bit 512 (8 unless CHECK and the block clips here or earlier).
-// `lut` must start on a 256-byte boundary of the shared window (aligned_smem):
-// the lookup address is the table base OR-ed with the next 8 stream bits.
+// `lkey` = lut_key() of the block's table: the lookup address is the key
+// XOR-ed with the next 8 stream bits.
 template <bool CHECK>
-__device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, const uint32_t* ws, int stride,
-                                            int& kv)
+__device__ __forceinline__ uint32_t decode8(Stream& st, uint32_t lkey, const uint32_t* ws, int stride, int& kv)
 {
     uint32_t nib = 0;
     int used = 0;
     kv = 0;
-    const uint32_t lut_sh = (uint32_t)__cvta_generic_to_shared(lut);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         refill(st, ws, stride);
@@ -108,8 +122,10 @@ __device__ __forceinline__ uint32_t decode8(Stream& st, const uint8_t* lut, cons
         int u = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            uint32_t e;  // the table is written before a CTA barrier: no ordering needed here
-            asm("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(lut_sh | (cur & 0xffu)));
+            // volatile with a memory clobber: the load stays on its side of
+            // the barriers around the tables' staging
+            uint32_t e;
+            asm volatile("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(lkey ^ (cur & 0xffu)) : "memory");
             uint32_t len = e >> 4;
             nib = __funnelshift_r(nib, e, 4);  // symbol into the top nibble; the first ends at the bottom
             cur >>= len;
@@ -138,20 +154,35 @@ __device__ __forceinline__ void mask_tail(uint32_t w[4], int kv)
 // Decodes one chunk into 4 bf16x2 words; also returns the nibbles.  The
 // lanes that run together take the checked walk as soon as one of them is
 // within 64 bits of the end (a vote), so a warp never runs both walks.
-__device__ __forceinline__ uint32_t chunk_values(Stream& st, const uint8_t* lut, const uint32_t* ws, int stride,
+__device__ __forceinline__ uint32_t chunk_values(Stream& st, uint32_t lkey, const uint32_t* ws, int stride,
                                                  const ValuePlanes& vp, uint32_t w[4])
 {
     int kv;
     uint32_t nib;
     if (__any_sync(__activemask(), st.room < 64))
-        nib = decode8<true>(st, lut, ws, stride, kv);
+        nib = decode8<true>(st, lkey, ws, stride, kv);
     else
-        nib = decode8<false>(st, lut, ws, stride, kv);
+        nib = decode8<false>(st, lkey, ws, stride, kv);
     uint32_t sh4 = nib << 4;
     planes_to_bf16<0>(vp, nib, sh4, w[0], w[1]);
     planes_to_bf16<1>(vp, nib, sh4, w[2], w[3]);
     if (kv < 8) mask_tail(w, kv);
     return nib;
+}
+
+// q / 127 correctly rounded (the outlier record's value, R15), without a
+// division: x0 = q * r with r = RN(1/127), the residual q - 127 x0 is exact
+// in one fused multiply-add, and one more gives the rounded quotient
+// (Markstein's correction step for division by a constant; checked against
+// the exactly rounded quotient for all 255 values of q, and bit-exact against
+// the oracle's IEEE division in the parity tests).
+__device__ __forceinline__ float q_over_127(int q)
+{
+    const float r = __uint_as_float(0x3c010204u);  // RN(1 / 127)
+    const float qf = (float)q;
+    const float x0 = __fmul_rn(qf, r);
+    const float res = __fmaf_rn(-x0, 127.0f, qf);
+    return __fmaf_rn(res, r, x0);
 }
 
 // Reads the 15-bit outlier record starting at stream bit `at` (>= 64).
@@ -217,6 +248,28 @@ __device__ __forceinline__ void stage_tables(const DevTables* tb, uint8_t* s_lut
             reinterpret_cast<uint4*>(s_lut)[i] = v[k];
         else if (i < kAll)
             reinterpret_cast<uint4*>(s_Ct)[i - kLutVec] = v[k];
+    }
+}
+
+// Copies a tensor's decode tables alone (65,536 B), every 16-byte load issued
+// before any store (kernels that read the centroids through the read-only
+// cache instead).
+template <int NT>
+__device__ __forceinline__ void stage_lut(const DevTables* tb, uint8_t* s_lut, int tid)
+{
+    constexpr int kLutVec = (int)(sizeof(((DevTables*)0)->lut) / 16);
+    constexpr int kPer = (kLutVec + NT - 1) / NT;
+    const uint4* lut = reinterpret_cast<const uint4*>(&tb->lut[0][0]);
+    uint4 v[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = tid + k * NT;
+        if (i < kLutVec) v[k] = __ldg(lut + i);
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = tid + k * NT;
+        if (i < kLutVec) reinterpret_cast<uint4*>(s_lut)[i] = v[k];
     }
 }
 

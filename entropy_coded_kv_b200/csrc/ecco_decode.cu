@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
             }
             stage_words(ws, kWordStride, q0, q1, q2, q3);
             const int p = (int)((q0.x >> 8) & 63u);
-            const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;  // table h * 64 + p
+            const uint32_t lkey = lut_key(s_lut, (q0.x >> 8) & 255u);  // table h * 64 + p
             const float s = __fmul_rn(S_t, e4m3_to_f32(code));
             const ValuePlanes vp = make_planes(s, s_Ct, p);
 
@@ -150,8 +150,8 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
 #pragma unroll 1
             for (int c = 0; c < G / 16; ++c) {  // 16 symbols, one 32-byte store each
                 uint32_t wa[4], wb[4];
-                chunk_values(st, lut, ws, kWordStride, vp, wa);
-                chunk_values(st, lut, ws, kWordStride, vp, wb);
+                chunk_values(st, lkey, ws, kWordStride, vp, wa);
+                chunk_values(st, lkey, ws, kWordStride, vp, wb);
                 if constexpr (kRows) {
                     *reinterpret_cast<uint4*>(row + 8 * c) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
                     *reinterpret_cast<uint4*>(row + 8 * c + 4) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
@@ -162,16 +162,15 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
 
             if (st.room >= 0) {  // unclipped: outlier records follow the codewords
                 // Each record is read at its own offset (independent loads,
-                // no chain through the stream window).  q / 127 is divided
-                // here (an ALU sequence) rather than looked up: the kernel is
-                // bound by the L1 data path, which a table gather would load
-                // further.
+                // no chain through the stream window); q / 127 by one
+                // correction step rather than a table gather, which would add
+                // to the L1 traffic.
                 const int n = min(kMaxRec, st.room / kRecBits);
                 const int at0 = kBlockBits - st.room;
                 for (int k = 0; k < n; ++k) {
                     const uint32_t rec = read_record(ws, kWordStride, at0 + k * kRecBits);
                     const int i = (int)(rec & (uint32_t)(G - 1));  // the 7-bit index, modulo G
-                    const float o = __fdiv_rn((float)(int)(int8_t)(uint8_t)(rec >> 7), 127.0f);
+                    const float o = q_over_127((int)(int8_t)(uint8_t)(rec >> 7));
                     const uint16_t v = (uint16_t)f32_to_bf16_bits(__fmul_rn(s, o));
                     if constexpr (kRows)
                         reinterpret_cast<uint16_t*>(row)[i] = v;
@@ -205,6 +204,8 @@ cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
     decode_kernel<WIDE, MAXSEG, G><<<grid, dec_threads<G>(), dec_smem<G>(), s>>>(P);
     return cudaGetLastError();
 }
+
+
 
 bool wide_ok(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 

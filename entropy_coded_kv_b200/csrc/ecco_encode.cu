@@ -39,7 +39,8 @@
 namespace ecco {
 namespace {
 
-constexpr int kEncWarps = 8;  // warps per CTA (16 groups in flight)
+constexpr int kEncWarps = 8;       // warps per CTA (16 groups in flight)
+constexpr int kEncCtasPerSm = 4;   // resident CTAs per SM (measured faster than 3 with 85 registers)
 constexpr int kRow = 97;      // words per pattern row: T[16] | lens4[16] | code[4][16] | pad
 constexpr int kRowLens = 16;
 constexpr int kRowCode = 32;
@@ -92,12 +93,23 @@ __device__ __forceinline__ void sort8_desc(uint32_t (&k)[8])
 #undef ECCO_CMPX
 }
 
-__device__ __forceinline__ int quantise(const uint32_t* R, float t7, float v)
+// 32-bit shared-window address of a word of the pattern rows.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// sym = number of thresholds T[0..13] of the row at shared address `R`
+// strictly below v (R9), by binary search: T[7] is in a register, the other
+// three levels read T[idx + 3], T[idx + 1], T[idx].
+__device__ __forceinline__ int quantise(uint32_t R, float t7, float v)
 {
     int idx = (t7 < v) ? 8 : 0;
-    idx += (__uint_as_float(R[idx + 3]) < v) ? 4 : 0;
-    idx += (__uint_as_float(R[idx + 1]) < v) ? 2 : 0;
-    idx += (__uint_as_float(R[idx]) < v) ? 1 : 0;
+    idx += (__uint_as_float(lds_u32(R + 4u * (uint32_t)idx + 12u)) < v) ? 4 : 0;
+    idx += (__uint_as_float(lds_u32(R + 4u * (uint32_t)idx + 4u)) < v) ? 2 : 0;
+    idx += (__uint_as_float(lds_u32(R + 4u * (uint32_t)idx)) < v) ? 1 : 0;
     return idx;
 }
 
@@ -117,9 +129,11 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
                      q.z & 0xffffu, q.z >> 16, q.w & 0xffffu, q.w >> 16};
     const int i0 = 8 * hl;
 
-    uint32_t key = 0;
+    // every element's key, kept for the outlier records
+    uint32_t kk[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) key = max(key, keyof(b[j], i0 + j));
+    for (int j = 0; j < 8; ++j) kk[j] = keyof(b[j], i0 + j);
+    uint32_t key = max(max(max(kk[0], kk[1]), max(kk[2], kk[3])), max(max(kk[4], kk[5]), max(kk[6], kk[7])));
     key = hw_max(gmask, key);
     if ((key >> 8) >= 0x7f80u) {  // a NaN or Inf in the group: encoded as +0, counted
         uint32_t nf = 0;
@@ -130,9 +144,9 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
                 ++nf;
             }
         cnt.nonfinite += hw_add(gmask, nf);
-        key = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) key = max(key, keyof(b[j], i0 + j));
+        for (int j = 0; j < 8; ++j) kk[j] = keyof(b[j], i0 + j);
+        key = max(max(max(kk[0], kk[1]), max(kk[2], kk[3])), max(max(kk[4], kk[5]), max(kk[6], kk[7])));
         key = hw_max(gmask, key);
     }
     const int m = 127 - (int)((key >> 1) & 127u);
@@ -152,17 +166,21 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     }
     const float inv = __ldg(&tb->inv_of_code[code]);
 
-    // ---- normalise; min / max over i != m (the scale element's slot takes a
-    // same-lane neighbour's value, which leaves both extremes alone)
+    // ---- normalise; min / max over i != m.  s carries x_m's sign, so u_m =
+    // |x_m| / |s| > 0 and no u_i exceeds it (|x_i| <= |x_m|, and rounding a
+    // product by the same factor keeps the order): u_m is the group's largest
+    // value, the minimum over i != m is the minimum over all i, and only the
+    // maximum has to leave slot m out.
     float u[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) u[j] = __fmul_rn(bf16_bits_to_f32(b[j]), inv);
-    float lmin, lmax;
+    const int jm = owner ? mj : 8;  // this lane's slot of m, if it has it
+    const float lmin = fminf(fminf(fminf(u[0], u[1]), fminf(u[2], u[3])), fminf(fminf(u[4], u[5]), fminf(u[6], u[7])));
+    float lmax;
     {
         float e[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) e[j] = (owner && j == mj) ? u[j ^ 1] : u[j];
-        lmin = fminf(fminf(fminf(e[0], e[1]), fminf(e[2], e[3])), fminf(fminf(e[4], e[5]), fminf(e[6], e[7])));
+        for (int j = 0; j < 8; ++j) e[j] = (j == jm) ? -INFINITY : u[j];
         lmax = fmaxf(fmaxf(fmaxf(e[0], e[1]), fmaxf(e[2], e[3])), fmaxf(fmaxf(e[4], e[5]), fmaxf(e[6], e[7])));
     }
     int p;
@@ -195,9 +213,9 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
         float best = 0.0f;
         p = 0;
         for (int q = 0; q < npat; ++q) {
-            const uint32_t* Rq = rows + q * kRow;
+            const uint32_t Rq = (uint32_t)__cvta_generic_to_shared(rows) + (uint32_t)(q * kRow) * 4u;
             const float* Cq = cent + q * 16;
-            const float tq = __uint_as_float(Rq[7]);
+            const float tq = __uint_as_float(lds_u32(Rq + 28u));
             float d2[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -216,14 +234,14 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     }
 
     // ---- quantise (count of thresholds strictly below u); lengths
-    const uint32_t* R = rows + p * kRow;
-    const float t7 = __uint_as_float(R[7]);
+    const uint32_t R = (uint32_t)__cvta_generic_to_shared(rows) + (uint32_t)(p * kRow) * 4u;
+    const float t7 = __uint_as_float(lds_u32(R + 28u));
     int sym[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sym[j] = (owner && j == mj) ? 15 : quantise(R, t7, u[j]);
+    for (int j = 0; j < 8; ++j) sym[j] = (j == jm) ? 15 : quantise(R, t7, u[j]);
     uint32_t acc = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc += R[kRowLens + sym[j]];
+    for (int j = 0; j < 8; ++j) acc += lds_u32(R + 4u * (uint32_t)(kRowLens + sym[j]));
     const uint32_t lo = hw_add(gmask, acc & 0x00ff00ffu);         // h = 0, 2
     const uint32_t hi = hw_add(gmask, (acc >> 8) & 0x00ff00ffu);  // h = 1, 3
     int h = 0, L = (int)(lo & 0xffffu);
@@ -232,7 +250,7 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
     if ((int)(hi >> 16) < L) { L = (int)(hi >> 16); h = 3; }
 
     // ---- two chunks of 4 codewords each, in stream order (<= 32 bits each)
-    const uint32_t* CW = R + kRowCode + 16 * h;
+    const uint32_t CW = R + 4u * (uint32_t)(kRowCode + 16 * h);
     uint32_t ch[2];
     int cl[2];
 #pragma unroll
@@ -241,7 +259,7 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
         int n = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            uint32_t e = CW[sym[4 * c + j]];
+            uint32_t e = lds_u32(CW + 4u * (uint32_t)sym[4 * c + j]);
             w |= (e & 0xffu) << n;
             n += (int)(e >> 8);
         }
@@ -278,7 +296,7 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
             // holds the element's bf16 bits and index, so nothing else is needed.
             uint32_t k[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) k[j] = (owner && j == mj) ? 0u : keyof(b[j], i0 + j) + 1u;
+            for (int j = 0; j < 8; ++j) k[j] = (j == jm) ? 0u : kk[j] + 1u;
             sort8_desc(k);
             for (int r = 0; r < n; ++r) {
                 const uint32_t bestk = hw_max(gmask, k[0]);
@@ -347,7 +365,7 @@ struct EncParams {  // by value: no device-side segment table
 // Each CTA encodes one contiguous, equal share of all groups of the launch,
 // segment by segment, restaging the pattern rows when it enters a new segment.
 template <int MAXSEG, int SEL, int G>
-__global__ void __launch_bounds__(kEncWarps * 32, 4) encode_kernel(const __grid_constant__ EncParams<MAXSEG> P)
+__global__ void __launch_bounds__(kEncWarps * 32, kEncCtasPerSm) encode_kernel(const __grid_constant__ EncParams<MAXSEG> P)
 {
     constexpr int kLanes = G / 8, kGpw = 32 / kLanes;  // lanes per group, groups per warp
     __shared__ uint32_t rows[kNPat * kRow];
@@ -439,7 +457,7 @@ cudaError_t run_encode(const EncParams<MAXSEG>& P, int select, cudaStream_t s)
 {
     const int per_cta = (32 / (G / 8)) * kEncWarps;
     int64_t want = (P.total + per_cta - 1) / per_cta;
-    int64_t cap = (int64_t)device_sm_count() * 4;  // resident CTAs at 4 per SM
+    int64_t cap = (int64_t)device_sm_count() * kEncCtasPerSm;  // one wave of resident CTAs
     int grid = (int)(want < cap ? want : cap);
     if (select == ECCO_SELECT_MSE)
         encode_kernel<MAXSEG, 1, G><<<grid, kEncWarps * 32, 0, s>>>(P);

@@ -7,25 +7,37 @@
 // (Review page, figure list: "Normalized Memory Requests for a GEMM Kernel" --
 // only compressed weights cross the memory bus.)
 //
-// CTA = 512 threads = 4 M-tiles of 128 rows; the CTA walks a range of column
-// groups, every thread decoding its own row's block (the block walker of
-// ecco_block.cuh).  Each 16 decoded values of a row (one K = 16 slice) go into
-// that tile's A buffer in shared memory (K-major, no swizzle: 8-row x 16-byte
-// core matrices); when the tile's 128 threads have written a slice, one
-// elected thread issues tcgen05.mma (M = 128, N = 16, K = 16, bf16 in, fp32
+// Work units are (row tile of 768 rows, one column group of 128 values); each
+// CTA (768 threads, one per SM) owns a balanced, contiguous range of units in
+// row-tile-major order, so consecutive units share a row tile and its
+// accumulators.  Thread t decodes row t's block of the unit with the block
+// walker of ecco_block.cuh; the CTA is 6 M-tiles of 128 rows (4 warps each).
+// Each 16 decoded values of a row (one K = 16 slice) go into that tile's A
+// buffer in shared memory (K-major, no swizzle: 8-row x 16-byte core
+// matrices); when the tile's 128 threads have written a slice, one elected
+// thread issues tcgen05.mma (M = 128, N = 16, K = 16, bf16 in, fp32
 // accumulate in tensor memory) and commits it to the buffer's mbarrier; the
 // buffer is written again only after that MMA completed.  A is double
 // buffered, so decoding the next slice overlaps the MMA of the current one.
-// x for the CTA's whole column range is staged once as the B operand.
+// x of the unit's column group is staged as the B operand (double buffered
+// by unit).  The centroids are read through the read-only cache; shared
+// memory holds the decode tables, the stream words, the decoded symbols (for
+// the records), A and B.
 //
 // Outlier records are known only at the end of a block's stream, after its
 // slices went to the tensor cores, so their effect is added on CUDA cores as
-// (new - old) * x.  Partial sums of column ranges are combined with fp32
-// atomics, as in the CUDA-core kernel.
+// (new - old) * x.  When a CTA's units move to the next row tile (and at the
+// end) each row's accumulators plus corrections are added to y with fp32
+// atomics (a row tile is split over a few CTAs).
 //
-// Every wait on an mbarrier is bounded; a wait that gives up increments a
-// device counter (ecco_device_timeouts) and the kernel finishes without
-// touching the buffer again.
+// Every wait on an mbarrier is bounded.  A wait that gives up counts itself
+// (ecco_device_timeouts) and raises a host-visible flag; its tile then issues
+// no more MMAs, the CTA agrees (a CTA-wide vote at the next unit) to stop and
+// to write nothing to y, waits once more (bounded) for the MMAs it already
+// committed, frees its tensor memory and returns.  The next tensor-core
+// ecco_decode_gemv call returns ECCO_ERR_TIMEOUT.
+#include <mutex>
+
 #include "ecco_block.cuh"
 
 namespace ecco {
@@ -34,22 +46,23 @@ __device__ unsigned int g_timeouts = 0;
 
 namespace {
 
-constexpr int kTcThreads = 512;
-constexpr int kTcTiles = kTcThreads / 128;
-constexpr int kTcStride = kTcThreads;        // word staging column stride
+constexpr int kTcThreads = 768;
+constexpr int kTcTiles = kTcThreads / 128;   // M-tiles of 128 rows
+constexpr int kTcStride = kTcThreads;        // word k of thread t's arrays at k * stride + t
 constexpr int kSliceBytes = 128 * 16 * 2;    // one 128 x 16 bf16 A slice
 constexpr int kBSliceBytes = 16 * 16 * 2;    // one 16 x 16 bf16 B slice
-constexpr int kMaxGroups = 8;                // column groups per CTA (x staged for all)
-constexpr uint32_t kSpinLimit = 1u << 22;  // polls; with the back-off below, well under a second
+constexpr int kBBytes = 8 * kBSliceBytes;    // x of one column group: 8 slices
+constexpr uint32_t kSpinLimit = 1u << 22;    // polls; with the back-off below, well under a second
 
 constexpr size_t kOffLut = 0;
-constexpr size_t kOffCt = kOffLut + 65536;
-constexpr size_t kOffWords = kOffCt + 4096;
-constexpr size_t kOffNib = kOffWords + 16 * kTcStride * 4;
-constexpr size_t kOffA = kOffNib + 16 * kTcThreads * 4;
+constexpr size_t kOffWords = kOffLut + 65536;
+constexpr size_t kOffNib = kOffWords + (size_t)16 * kTcStride * 4;
+constexpr size_t kOffA = kOffNib + (size_t)16 * kTcThreads * 4;
 constexpr size_t kOffB = kOffA + (size_t)kTcTiles * 2 * kSliceBytes;
-constexpr size_t kOffBar = kOffB + (size_t)kMaxGroups * 8 * kBSliceBytes;
-constexpr size_t kTcSmem = kOffBar + 128 + kSmemAlign;
+constexpr size_t kOffBar = kOffB + (size_t)2 * kBBytes;
+constexpr int kNumBars = 3 * kTcTiles;  // [tile][2] A buffers, then done[tile]
+constexpr size_t kTcSmem = kOffBar + (size_t)kNumBars * 8 + 16 + kSmemAlign;
+constexpr uint32_t kTmemCols = 128;     // 6 tiles x 16 fp32 columns, rounded to a power of 2
 
 // Instruction descriptor: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12
 // = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -76,8 +89,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
 
 // Waits for the phase with the given parity to complete: non-blocking polls,
 // with a short sleep after the first few, at most kSpinLimit of them.
-// Returns false (and counts a timeout) if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+// Returns false if it gave up, after counting the timeout and raising `flag`
+// (host-visible) when there is one.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flag)
 {
     const uint32_t a = smem_u32(bar);
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
@@ -93,12 +107,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
         if (i >= 16) __nanosleep(64);
     }
     atomicAdd(&g_timeouts, 1u);
+    if (flag) {
+        *reinterpret_cast<volatile int*>(flag) = 1;
+        __threadfence_system();
+    }
     return false;
 }
 
-__device__ __forceinline__ void named_sync(int id, int n)
+// Named barrier over the n threads of a tile that also ANDs a flag across them.
+__device__ __forceinline__ bool tile_sync_and(int id, int n, bool v)
 {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0u;
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
@@ -124,59 +152,60 @@ __device__ __forceinline__ uint32_t a_offset(int row, int khalf)
     return (uint32_t)((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
-    gemm_tc_kernel(const DevTables* __restrict__ tb, const uint8_t* __restrict__ blocks, int64_t rows,
-                   int64_t gpr, const uint16_t* __restrict__ x, int batch, int64_t cols, int splits,
-                   float* __restrict__ y)
+// Byte offset of x[b][k] (k within a 16-wide slice) inside a 16 x 16 B slice.
+__device__ __forceinline__ uint32_t b_offset(int b, int kk)
+{
+    return (uint32_t)((b >> 3) * 256 + (kk >> 3) * 128 + (b & 7) * 16 + (kk & 7) * 2);
+}
+
+struct TcArgs {
+    const DevTables* tb;
+    const uint8_t* blocks;
+    const uint16_t* x;
+    float* y;
+    int* flag;  // host-visible timeout flag (mapped pinned memory), or null
+    int64_t rows, gpr, cols, units;
+    int batch;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_constant__ TcArgs A)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t* smem = aligned_smem(smem_raw);
     uint8_t* s_lut = smem + kOffLut;
-    float* s_Ct = reinterpret_cast<float*>(smem + kOffCt);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kOffWords);
     uint32_t* s_nib = reinterpret_cast<uint32_t*>(smem + kOffNib);
     uint8_t* s_A = smem + kOffA;
     uint8_t* s_B = smem + kOffB;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);  // [tile][2] then done[tile]
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + 96);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tile = warp >> 2;             // 4 warps per 128-row tile
+    const int tile = warp >> 2;               // 4 warps per 128-row tile
     const int trow = (warp & 3) * 32 + lane;  // row inside the tile = TMEM lane
+    const DevTables* tb = A.tb;
+    const float* Ct = &tb->Ct[0][0];
 
-    // this CTA's column groups
-    const int64_t g_begin = gpr * blockIdx.y / splits, g_end = gpr * (blockIdx.y + 1) / splits;
-    const int ng = (int)(g_end - g_begin);
+    const int64_t u0 = A.units * blockIdx.x / gridDim.x, u1 = A.units * (blockIdx.x + 1) / gridDim.x;
 
-    stage_tables<kTcThreads>(tb, s_lut, s_Ct, tid);
-    // B: x[b][k] for the column range, as ng * 8 slices of 16 x 16, K-major
-    for (int e = tid; e < ng * 128 * 16; e += kTcThreads) {
-        const int b = e & 15, k = e >> 4;  // k within the range
-        uint16_t v = 0;
-        if (b < batch) v = x[(int64_t)b * cols + g_begin * kG + k];
-        const int slice = k >> 4, kk = k & 15;
-        const uint32_t off = slice * kBSliceBytes + (b >> 3) * 256 + (kk >> 3) * 128 + (b & 7) * 16 + (kk & 7) * 2;
-        *reinterpret_cast<uint16_t*>(s_B + off) = v;
-    }
+    stage_lut<kTcThreads>(tb, s_lut, tid);
     if (tid == 0) {
-        for (int i = 0; i < 3 * kTcTiles; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
-                     "r"(64)
+                     "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // B staged by generic stores
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem_d = *s_tmem + (uint32_t)(16 * tile);  // this tile's 16 fp32 columns
+    const uint32_t taddr = tmem_d + ((uint32_t)((warp & 3) * 32) << 16);
     const float S_t = tb->S_t;
 
-    const int64_t row = (int64_t)blockIdx.x * kTcThreads + tile * 128 + trow;
-    const bool row_ok = row < rows;
     uint32_t* ws = s_w + tid;
     uint32_t* nibs = s_nib + tid;
     uint8_t* A0 = s_A + tile * 2 * kSliceBytes;
@@ -186,13 +215,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float corr[16];
 #pragma unroll
     for (int b = 0; b < 16; ++b) corr[b] = 0.0f;
-    bool ok = true;
-    int t = 0;  // slice counter over the CTA's column range
+    bool ok = true;      // uniform in the tile after every slice, in the CTA after every unit start
+    int t = 0;           // slices of this tile so far (its A buffer is t & 1)
+    int flushes = 0;     // completed phases of bar_done
+    bool acc = false;    // the tile's accumulators hold a partial sum
+    int64_t tile_row = (u0 < u1) ? u0 / A.gpr : 0;
 
-    for (int gi = 0; gi < ng; ++gi) {
+    // Adds each thread's row of its tile's accumulators (plus the record
+    // corrections) to y and starts the next row tile from zero.  Called by
+    // every thread at the same points.
+    auto flush = [&](int64_t rt) {
+        if (issuer && ok && acc) mma_commit(bar_done);
+        if (ok && acc) ok = mbar_wait(bar_done, (uint32_t)(flushes & 1), A.flag);
+        ok = __syncthreads_and(ok);
+        if (acc) ++flushes;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+            "[%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        const int64_t row = rt * kTcThreads + tid;
+        if (ok && acc && row < A.rows) {
+#pragma unroll
+            for (int b = 0; b < 16; ++b)
+                if (b < A.batch) atomicAdd(&A.y[(int64_t)b * A.rows + row], __uint_as_float(v[b]) + corr[b]);
+        }
+#pragma unroll
+        for (int b = 0; b < 16; ++b) corr[b] = 0.0f;
+        acc = false;
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    };
+
+    for (int64_t u = u0; u < u1; ++u) {
+        const int64_t rt = u / A.gpr, g = u - rt * A.gpr;
+        if (rt != tile_row) {
+            flush(tile_row);
+            tile_row = rt;
+        }
+        // ---- x of this column group as the B operand (buffer u & 1), once
+        // every MMA that read the buffer (unit u - 2) has completed: the
+        // tile's slice t - 2 completes after them; then the CTA agrees
+        uint8_t* B = s_B + (int)(u & 1) * kBBytes;
+        if (t >= 2 && ok) ok = mbar_wait(&bar_buf[t & 1], (uint32_t)(((t >> 1) - 1) & 1), A.flag);
+        ok = __syncthreads_and(ok);
+        if (!ok) break;  // CTA-uniform
+        for (int e = tid; e < 16 * kG; e += kTcThreads) {
+            const int b = e & 15, k = e >> 4;
+            const uint16_t v = (b < A.batch) ? A.x[(int64_t)b * A.cols + g * kG + k] : (uint16_t)0;
+            *reinterpret_cast<uint16_t*>(B + (k >> 4) * kBSliceBytes + b_offset(b, k & 15)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // B written by generic stores
+        __syncthreads();
+
+        // ---- this thread's row block
+        const int64_t row = rt * kTcThreads + tid;
+        const bool row_ok = row < A.rows;
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, q2 = q0, q3 = q0;
         if (row_ok) {
-            const uint8_t* src = blocks + (row * gpr + g_begin + gi) * ECCO_BLOCK_BYTES;
+            const uint8_t* src = A.blocks + (row * A.gpr + g) * ECCO_BLOCK_BYTES;
             q0 = ldg_nc_v4(src);
             q1 = ldg_nc_v4(src + 16);
             q2 = ldg_nc_v4(src + 32);
@@ -200,33 +284,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         const uint32_t code = q0.x & 0xffu;
         const int p = (int)((q0.x >> 8) & 63u);
+        // a row past the end or a null scale contributes zeros
         const float s = (row_ok && !scale_code_is_null(code)) ? __fmul_rn(S_t, e4m3_to_f32(code)) : 0.0f;
         stage_words(ws, kTcStride, q0, q1, q2, q3);
-        const ValuePlanes vp = make_planes(s, s_Ct, p);
-        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
+        const ValuePlanes vp = make_planes<true>(s, Ct, p);
+        const uint32_t lkey = lut_key(s_lut, (q0.x >> 8) & 255u);
         Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 
 #pragma unroll 1
         for (int sl = 0; sl < 8; ++sl, ++t) {
             uint32_t wa[4], wb[4];
-            nibs[(2 * sl) * kTcThreads] = chunk_values(st, lut, ws, kTcStride, vp, wa);
-            nibs[(2 * sl + 1) * kTcThreads] = chunk_values(st, lut, ws, kTcStride, vp, wb);
+            nibs[(2 * sl) * kTcThreads] = chunk_values(st, lkey, ws, kTcStride, vp, wa);
+            nibs[(2 * sl + 1) * kTcThreads] = chunk_values(st, lkey, ws, kTcStride, vp, wb);
             const int buf = t & 1, use = t >> 1;
-            if (use >= 1 && ok) ok = mbar_wait(&bar_buf[buf], (uint32_t)((use - 1) & 1));
-            uint8_t* A = A0 + buf * kSliceBytes;
-            if (ok) {
-                *reinterpret_cast<uint4*>(A + a_offset(trow, 0)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                *reinterpret_cast<uint4*>(A + a_offset(trow, 1)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-            }
+            if (use >= 1 && ok) ok = mbar_wait(&bar_buf[buf], (uint32_t)((use - 1) & 1), A.flag);
+            uint8_t* Ab = A0 + buf * kSliceBytes;
+            *reinterpret_cast<uint4*>(Ab + a_offset(trow, 0)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            *reinterpret_cast<uint4*>(Ab + a_offset(trow, 1)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            named_sync(1 + tile, 128);
+            // the tile's 128 rows are written and its threads agree that no wait gave up
+            ok = tile_sync_and(1 + tile, 128, ok);
             if (issuer && ok) {
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint64_t ad = smem_desc(smem_u32(A));
-                const uint64_t bd = smem_desc(smem_u32(s_B + (gi * 8 + sl) * kBSliceBytes));
-                mma_bf16(tmem_d, ad, bd, t > 0 ? 1u : 0u);
+                const uint64_t ad = smem_desc(smem_u32(Ab));
+                const uint64_t bd = smem_desc(smem_u32(B + sl * kBSliceBytes));
+                mma_bf16(tmem_d, ad, bd, acc ? 1u : 0u);
                 mma_commit(&bar_buf[buf]);
             }
+            acc = true;
         }
 
         if (s != 0.0f && st.room >= 0) {  // outlier records: add (new - old) * x
@@ -236,8 +321,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // already seen (128-bit mask) is skipped.
             uint32_t seen0 = 0u, seen1 = 0u, seen2 = 0u, seen3 = 0u;
             for (int k = n - 1; k >= 0; --k) {
-                uint32_t rec = read_record(ws, kTcStride, at0 + k * kRecBits);
-                int i = (int)(rec & 127u);
+                const uint32_t rec = read_record(ws, kTcStride, at0 + k * kRecBits);
+                const int i = (int)(rec & 127u);
                 const uint32_t bit = 1u << (i & 31), q = (uint32_t)i >> 5;
                 const uint32_t was = (q == 0u ? seen0 : q == 1u ? seen1 : q == 2u ? seen2 : seen3) & bit;
                 seen0 |= (q == 0u) ? bit : 0u;
@@ -245,51 +330,72 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 seen2 |= (q == 2u) ? bit : 0u;
                 seen3 |= (q == 3u) ? bit : 0u;
                 if (was) continue;
-                float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, __ldg(&tb->o_of_q[rec >> 7]))));
-                uint32_t osym = (nibs[(i >> 3) * kTcThreads] >> (4 * (i & 7))) & 15u;
-                uint32_t ow = (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);
-                uint32_t oh = (osym < 8) ? ((osym < 4) ? vp.hi[0] : vp.hi[1]) : ((osym < 12) ? vp.hi[2] : vp.hi[3]);
-                uint32_t sh = 8 * (osym & 3);
-                float ov = __uint_as_float((((ow >> sh) & 0xffu) | (((oh >> sh) & 0xffu) << 8)) << 16);
-                float dv = nv - ov;
-                const int sl = i >> 4, kk = i & 15;
-                const uint8_t* Bs = s_B + (gi * 8 + sl) * kBSliceBytes + (kk >> 3) * 128 + (kk & 7) * 2;
+                const float nv =
+                    bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, q_over_127((int)(int8_t)(uint8_t)(rec >> 7)))));
+                const uint32_t osym = (nibs[(i >> 3) * kTcThreads] >> (4 * (i & 7))) & 15u;
+                const uint32_t ow =
+                    (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);
+                const uint32_t oh =
+                    (osym < 8) ? ((osym < 4) ? vp.hi[0] : vp.hi[1]) : ((osym < 12) ? vp.hi[2] : vp.hi[3]);
+                const uint32_t sh = 8 * (osym & 3);
+                const float ov = __uint_as_float((((ow >> sh) & 0xffu) | (((oh >> sh) & 0xffu) << 8)) << 16);
+                const float dv = nv - ov;
+                const uint8_t* Bs = B + (i >> 4) * kBSliceBytes;
 #pragma unroll
                 for (int b = 0; b < 16; ++b) {
-                    float xv = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(Bs + (b >> 3) * 256 + (b & 7) * 16));
+                    const float xv = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(Bs + b_offset(b, i & 15)));
                     corr[b] = fmaf(dv, xv, corr[b]);
                 }
             }
         }
     }
+    flush(tile_row);  // every thread leaves the unit loop at the same unit
 
-    // all MMAs of this tile done -> read the accumulator rows
-    if (issuer && ok) mma_commit(bar_done);
-    if (ok && t > 0) ok = mbar_wait(bar_done, 0u);
-    __syncwarp();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    uint32_t v[16];
-    const uint32_t taddr = tmem_d + ((uint32_t)((warp & 3) * 32) << 16);
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-    if (row_ok && ok && t > 0) {
-#pragma unroll
-        for (int b = 0; b < 16; ++b)
-            if (b < batch) atomicAdd(&y[(int64_t)b * rows + row], __uint_as_float(v[b]) + corr[b]);
-    }
+    // before the tensor memory is freed: the MMAs this tile committed are
+    // done (bounded once more if a wait already gave up)
+    if (t >= 1) mbar_wait(&bar_buf[(t - 1) & 1], (uint32_t)(((t - 1) >> 1) & 1), nullptr);
+    if (t >= 2) mbar_wait(&bar_buf[t & 1], (uint32_t)(((t >> 1) - 1) & 1), nullptr);
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem), "r"(64) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem), "r"(kTmemCols)
+                     : "memory");
 }
+
+// Waits on an mbarrier that nothing arrives at, with the pipeline's bounded
+// wait: it gives up, counts the timeout and raises the flag.
+__global__ void wait_timeout_selftest_kernel(int* flag)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_wait(&bar, 0u, flag);
+    }
+}
+
+std::once_flag g_flag_once;
+int* g_flag = nullptr;  // mapped pinned int shared by all devices; null if it could not be allocated
 
 }  // namespace
 
-size_t gemm_tc_smem() { return kTcSmem; }
+int* timeout_flag()
+{
+    std::call_once(g_flag_once, [] {
+        void* p = nullptr;
+        if (cudaHostAlloc(&p, sizeof(int), cudaHostAllocMapped | cudaHostAllocPortable) == cudaSuccess) {
+            *static_cast<volatile int*>(p) = 0;
+            g_flag = static_cast<int*>(p);
+        }
+    });
+    return g_flag;
+}
+
+bool timeout_raised()
+{
+    int* f = timeout_flag();
+    return f && *reinterpret_cast<volatile int*>(f) != 0;
+}
 
 cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                            const uint16_t* x, int batch, float* y, cudaStream_t s)
@@ -299,14 +405,26 @@ cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t 
         return e0;
     cudaError_t e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)batch * (size_t)rows, s);
     if (e != cudaSuccess) return e;
-    const int64_t gpr = cols / kG;
-    const int64_t chunks = (rows + kTcThreads - 1) / kTcThreads;
-    int64_t splits = (int64_t)device_sm_count() / chunks;  // one wave of CTAs
-    if (splits < (gpr + kMaxGroups - 1) / kMaxGroups) splits = (gpr + kMaxGroups - 1) / kMaxGroups;
-    if (splits > gpr) splits = gpr;
-    if (splits < 1) splits = 1;
-    dim3 grid((unsigned)chunks, (unsigned)splits);
-    gemm_tc_kernel<<<grid, kTcThreads, kTcSmem, s>>>(t->d, blocks, rows, gpr, x, batch, cols, (int)splits, y);
+    TcArgs A;
+    A.tb = t->d;
+    A.blocks = blocks;
+    A.x = x;
+    A.y = y;
+    A.flag = timeout_flag();
+    A.rows = rows;
+    A.gpr = cols / kG;
+    A.cols = cols;
+    A.units = (rows + kTcThreads - 1) / kTcThreads * A.gpr;
+    A.batch = batch;
+    const int64_t sms = device_sm_count();
+    const int grid = (int)(A.units < sms ? A.units : sms);  // one resident CTA per SM, balanced unit ranges
+    gemm_tc_kernel<<<grid, kTcThreads, kTcSmem, s>>>(A);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_selftest(cudaStream_t s)
+{
+    wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(timeout_flag());
     return cudaGetLastError();
 }
 
@@ -315,5 +433,7 @@ cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t 
 extern "C" int ecco_device_timeouts(unsigned int* out)
 {
     if (!out) return ECCO_ERR_ARG;
-    return cudaMemcpyFromSymbol(out, ecco::g_timeouts, sizeof(unsigned int)) == cudaSuccess ? ECCO_OK : ECCO_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(out, ecco::g_timeouts, sizeof(unsigned int)) != cudaSuccess) return ECCO_ERR_CUDA;
+    if (int* f = ecco::timeout_flag()) *reinterpret_cast<volatile int*>(f) = 0;
+    return ECCO_OK;
 }

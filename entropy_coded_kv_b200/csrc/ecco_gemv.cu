@@ -112,13 +112,13 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
         const float s = (row_ok && !scale_code_is_null(code)) ? __fmul_rn(S_t, e4m3_to_f32(code)) : 0.0f;
         stage_words(ws, kGvStride, q0, q1, q2, q3);
         const ValuePlanes vp = make_planes(s, s_Ct, p);
-        const uint8_t* lut = s_lut + ((q0.x >> 8) & 255u) * 256;
+        const uint32_t lkey = lut_key(s_lut, (q0.x >> 8) & 255u);
 
         Stream st{q0.x, q0.y, kHdrBits, 2, kPayloadBits};
 #pragma unroll 1
         for (int c = 0; c < 16; ++c) {
             uint32_t w[4];
-            nibs[c * kGvThreads] = chunk_values(st, lut, ws, kGvStride, vp, w);
+            nibs[c * kGvThreads] = chunk_values(st, lkey, ws, kGvStride, vp, w);
             // the chunk's 8 x B inputs as 16-byte broadcast loads (one L1 wavefront each)
             float xk[8 * B];
 #pragma unroll

@@ -42,7 +42,9 @@ struct DevTables {
     float2 ends[kNPat];             // (C[p][0], C[p][14])
     uint32_t lens4[kNPat][16];      // byte h = length of symbol s in codebook h
     uint32_t code[kNPat][kNBook][16];  // bits 0-7 codeword in stream order, bits 8-11 length
-    uint8_t lut[kNBook * kNPat][256];  // [h * 64 + p] (= header bits 8-15): next 8 stream bits -> symbol | length << 4
+    // [t = h * 64 + p] (= header bits 8-15): the next 8 stream bits e -> symbol | length << 4, entry e at
+    // byte e ^ ((t & 31) << 2) (word-level swizzle against bank conflicts, see lut_key)
+    uint8_t lut[kNBook * kNPat][256];
     // Scale tables, filled on the device at creation with the same operations
     // the encoder would otherwise run per group (IEEE divide, E4M3 rounding,
     // fp32 multiply, correctly rounded reciprocal):
@@ -73,6 +75,11 @@ cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t row
 cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                            const uint16_t* x, int batch, float* y, cudaStream_t s);
 cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s);
+// Timeouts of the tensor-core pipeline's bounded waits: a host-visible flag
+// (mapped pinned memory, allocated once) that a wait which gave up raises.
+int* timeout_flag();
+bool timeout_raised();
+cudaError_t launch_wait_timeout_selftest(cudaStream_t s);
 // Activation format: 64-value groups (the descriptor counts 64-value groups).
 cudaError_t launch_encode_act(const ecco_tables* t, const uint16_t* x, const ecco_desc& d,
                               uint8_t* blocks, ecco_stats* stats, cudaStream_t s);

@@ -96,14 +96,15 @@ void derive(const Blob& b, DevTables* t)
         for (int h = 0; h < kNBook; ++h) {
             uint32_t code[kNSym];
             canonical(b.len[p][h], code);
-            uint8_t* lut = t->lut[h * kNPat + p];
+            const uint32_t tix = (uint32_t)(h * kNPat + p);
+            uint8_t one[256];  // next 8 stream bits -> symbol | length << 4, unswizzled
             for (int s = 0; s < kNSym; ++s) {
                 int l = b.len[p][h][s];
                 uint32_t rev = reverse_bits(code[s], l);
                 t->code[p][h][s] = rev | ((uint32_t)l << 8);
-                for (uint32_t tail = 0; tail < (1u << (8 - l)); ++tail)
-                    lut[rev | (tail << l)] = (uint8_t)(s | (l << 4));
+                for (uint32_t tail = 0; tail < (1u << (8 - l)); ++tail) one[rev | (tail << l)] = (uint8_t)(s | (l << 4));
             }
+            for (uint32_t e = 0; e < 256; ++e) t->lut[tix][e ^ ((tix & 31u) << 2)] = one[e];
         }
     }
 }
@@ -146,6 +147,7 @@ extern "C" int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables**
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ECCO_ERR_CUDA;
     if (prop.major != 10) return ECCO_ERR_UNSUPPORTED;
 
+    timeout_flag();  // the tensor-core pipeline's timeout flag, allocated once, off the hot path
     DevTables* host = new (std::nothrow) DevTables;
     if (!host) return ECCO_ERR_ARG;
     derive(b, host);

@@ -295,9 +295,21 @@ int ecco_huffman_lengths(const double* weights, int n, int max_len, uint8_t* len
 
 /* Number of bounded device-side waits (tensor-core decode+GEMV pipeline) that
  * gave up since the library was loaded on the current device; 0 in normal
- * operation.  A kernel whose wait gives up skips the rest of its work instead
- * of hanging, so its outputs are incomplete.  Blocking (reads device memory). */
+ * operation.  A CTA whose wait gives up stops issuing tensor-core work, adds
+ * nothing to y and returns instead of hanging, so that launch's y is
+ * incomplete.  Because launches are asynchronous, the failure is reported
+ * like CUDA's own asynchronous errors: it raises a host-visible flag, and
+ * every later ecco_decode_gemv call with batch > 4 returns ECCO_ERR_TIMEOUT
+ * (enqueuing nothing) until this function is called, which reads the count
+ * and clears the flag.  Blocking (reads device memory). */
+#define ECCO_ERR_TIMEOUT (-8) /* a bounded device wait gave up in an earlier launch */
 int ecco_device_timeouts(unsigned int* out);
+
+/* Diagnostic for the timeout path above, with no fault and no hang: launches
+ * one kernel that waits, with the pipeline's bounded wait (well under a
+ * second), on an mbarrier that nothing completes, so the wait gives up,
+ * counts itself and raises the flag.  Asynchronous on `stream`. */
+int ecco_selftest_wait_timeout(void* stream);
 
 const char* ecco_strerror(int code);
 int ecco_abi_version(void);

@@ -41,13 +41,13 @@ def test_header_constants_match_binding(lib):
     assert f"ECCO_TABLES_BYTES {_lib.TABLES_BYTES}u" in src
     consts = {m.group(1): m.group(2) for m in re.finditer(r"#define (ECCO_\w+) \(?(-?[0-9x]+)", src)}
     for name in ("OK", "ERR_ARG", "ERR_ALIGN", "ERR_TABLES", "ERR_CUDA", "ERR_DEVICE", "ERR_UNSUPPORTED",
-                 "ERR_WORKSPACE", "SELECT_MINMAX", "SELECT_MSE"):
+                 "ERR_WORKSPACE", "ERR_TIMEOUT", "SELECT_MINMAX", "SELECT_MSE"):
         assert int(consts["ECCO_" + name], 0) == getattr(_lib, "ECCO_" + name if name.startswith(("OK", "ERR")) else name), name
     assert "ECCO_ATTENTION_STATIC_WS_BYTES (4u << 20)" in src and _lib.ATTENTION_STATIC_WS_BYTES == 4 << 20
     assert int(consts["ECCO_MAX_SEGMENTS"]) == _lib.MAX_SEGMENTS
     assert int(consts["ECCO_GROUP"]) == ecco.GROUP and int(consts["ECCO_GROUP_ACT"]) == ecco.GROUP_ACT
     assert lib.ecco_abi_version() == 1
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
         assert _lib.strerror(code)
 
 

@@ -389,10 +389,19 @@ def test_tensor_core_gemv_one_hot_columns_are_exact(batch):
 
 
 def test_no_device_wait_gave_up():
+    """Tensor-core GEMV launches leave the timeout count where it was."""
     import ctypes
-    n = ctypes.c_uint(123)
-    assert _lib.load().ecco_device_timeouts(ctypes.byref(n)) == 0
-    assert n.value == 0
+    lib = _lib.load()
+    before, after = ctypes.c_uint(123), ctypes.c_uint(456)
+    assert lib.ecco_device_timeouts(ctypes.byref(before)) == 0
+    blob = table_set("learned_w")
+    t = ecco.Tables(blob, DEV)
+    blocks = torch.from_numpy(oracle.encode(blob, inputs("t5", 700 * 3, seed=2), nthreads=8)[0]).to(DEV)
+    for batch in (5, 16):
+        ecco.decode_gemv(blocks, t, 700, 384, W.activations(384, batch, device=DEV))
+    torch.cuda.synchronize()
+    assert lib.ecco_device_timeouts(ctypes.byref(after)) == 0
+    assert after.value == before.value
 
 
 def test_offsets_past_4_gib():
