@@ -11,18 +11,25 @@
 // CTA (768 threads, one per SM) owns a balanced, contiguous range of units in
 // row-tile-major order, so consecutive units share a row tile and its
 // accumulators.  Thread t decodes row t's block of the unit with the block
-// walker of ecco_block.cuh; the CTA is 6 M-tiles of 128 rows (4 warps each).
-// Each 16 decoded values of a row (one K = 16 slice) go into that tile's A
-// buffer in shared memory (K-major, no swizzle: 8-row x 16-byte core
-// matrices); when the tile's 128 threads have written a slice, one elected
-// thread issues tcgen05.mma (M = 128, N = 16, K = 16, bf16 in, fp32
-// accumulate in tensor memory) and commits it to the buffer's mbarrier; the
-// buffer is written again only after that MMA completed.  A is double
-// buffered, so decoding the next slice overlaps the MMA of the current one.
-// x of the unit's column group is staged as the B operand (double buffered
-// by unit).  The centroids are read through the read-only cache; shared
-// memory holds the decode tables, the stream words, the decoded symbols (for
-// the records), A and B.
+// walker of ecco_block.cuh.  The walk's speed comes from the warps running
+// freely (its latency is hidden by the other warps), so every warp feeds the
+// tensor cores on its own, with no barrier between warps inside a unit:
+//   - the 4 warps w = 4j..4j+3 share A tile buffers j (double buffered), 128
+//     rows x 16 values (one K = 16 slice, K-major, no swizzle: 8-row x
+//     16-byte core matrices); warp w writes rows 32 (w & 3) .. + 31;
+//   - lane 0 of warp w then issues tcgen05.mma (M = 128, N = 16, K = 16, bf16
+//     in, fp32 accumulate) on the whole tile into warp w's own 16 columns of
+//     tensor memory, and commits it to the warp's mbarrier for that buffer;
+//   - row r of the product depends on row r of A only, so the rows the other
+//     three warps are writing (or have overwritten) reach only lanes of warp
+//     w's columns that warp w never reads: it reads back lanes 32 (w & 3) ..
+//     + 31, the lanes its own rows produced;
+//   - a warp writes a buffer again only after its own MMA that read it has
+//     completed.
+// x of the unit's column group is the B operand (double buffered by unit:
+// a CTA barrier per unit).  The centroids are read through the read-only
+// cache; shared memory holds the decode tables, the stream words, the decoded
+// symbols (for the records), A and B.
 //
 // Outlier records are known only at the end of a block's stream, after its
 // slices went to the tensor cores, so their effect is added on CUDA cores as
@@ -31,11 +38,12 @@
 // atomics (a row tile is split over a few CTAs).
 //
 // Every wait on an mbarrier is bounded.  A wait that gives up counts itself
-// (ecco_device_timeouts) and raises a host-visible flag; its tile then issues
-// no more MMAs, the CTA agrees (a CTA-wide vote at the next unit) to stop and
-// to write nothing to y, waits once more (bounded) for the MMAs it already
-// committed, frees its tensor memory and returns.  The next tensor-core
-// ecco_decode_gemv call returns ECCO_ERR_TIMEOUT.
+// (ecco_device_timeouts) and raises a host-visible flag; the warp then issues
+// no more MMAs, the CTA agrees (a CTA-wide vote at the next unit and at every
+// accumulator read-out) to stop and to write nothing to y, waits once more
+// (bounded) for the MMAs it already committed, frees its tensor memory and
+// returns.  The next tensor-core ecco_decode_gemv call returns
+// ECCO_ERR_TIMEOUT.
 #include <mutex>
 
 #include "ecco_block.cuh"
@@ -60,9 +68,10 @@ constexpr size_t kOffNib = kOffWords + (size_t)16 * kTcStride * 4;
 constexpr size_t kOffA = kOffNib + (size_t)16 * kTcThreads * 4;
 constexpr size_t kOffB = kOffA + (size_t)kTcTiles * 2 * kSliceBytes;
 constexpr size_t kOffBar = kOffB + (size_t)2 * kBBytes;
-constexpr int kNumBars = 3 * kTcTiles;  // [tile][2] A buffers, then done[tile]
+constexpr int kTcWarps = kTcThreads / 32;
+constexpr int kNumBars = 2 * kTcWarps;  // [warp][2]: the warp's MMAs on A buffer 0 / 1
 constexpr size_t kTcSmem = kOffBar + (size_t)kNumBars * 8 + 16 + kSmemAlign;
-constexpr uint32_t kTmemCols = 128;     // 6 tiles x 16 fp32 columns, rounded to a power of 2
+constexpr uint32_t kTmemCols = 512;     // 24 warps x 16 fp32 columns, rounded up to a power of 2
 
 // Instruction descriptor: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12
 // = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -112,21 +121,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* f
         __threadfence_system();
     }
     return false;
-}
-
-// Named barrier over the n threads of a tile that also ANDs a flag across them.
-__device__ __forceinline__ bool tile_sync_and(int id, int n, bool v)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(id), "r"(n)
-        : "memory");
-    return r != 0u;
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
@@ -202,33 +196,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const uint32_t tmem_d = *s_tmem + (uint32_t)(16 * tile);  // this tile's 16 fp32 columns
-    const uint32_t taddr = tmem_d + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t tmem_d = *s_tmem + (uint32_t)(16 * warp);  // this warp's 16 fp32 columns
+    const uint32_t taddr = tmem_d + ((uint32_t)((warp & 3) * 32) << 16);  // ... at its own lanes
     const float S_t = tb->S_t;
 
     uint32_t* ws = s_w + tid;
     uint32_t* nibs = s_nib + tid;
     uint8_t* A0 = s_A + tile * 2 * kSliceBytes;
-    const bool issuer = (warp & 3) == 0 && lane == 0;
-    uint64_t* bar_buf = &bars[tile * 2];
-    uint64_t* bar_done = &bars[2 * kTcTiles + tile];
+    const bool issuer = lane == 0;
+    uint64_t* bar_buf = &bars[warp * 2];
     float corr[16];
 #pragma unroll
     for (int b = 0; b < 16; ++b) corr[b] = 0.0f;
-    bool ok = true;      // uniform in the tile after every slice, in the CTA after every unit start
-    int t = 0;           // slices of this tile so far (its A buffer is t & 1)
-    int flushes = 0;     // completed phases of bar_done
-    bool acc = false;    // the tile's accumulators hold a partial sum
+    bool ok = true;      // uniform in the warp after every slice, in the CTA after every unit start
+    int t = 0;           // slices so far (the A buffer is t & 1)
+    bool acc = false;    // the warp's accumulators hold a partial sum
     int64_t tile_row = (u0 < u1) ? u0 / A.gpr : 0;
 
-    // Adds each thread's row of its tile's accumulators (plus the record
+    // Waits until this warp's MMAs issued so far have completed (the commit of
+    // the last slice completes after all of them).
+    auto drain = [&]() {
+        if (t >= 1 && ok) ok = mbar_wait(&bar_buf[(t - 1) & 1], (uint32_t)(((t - 1) >> 1) & 1), A.flag);
+    };
+    // Adds each thread's row of its warp's accumulators (plus the record
     // corrections) to y and starts the next row tile from zero.  Called by
     // every thread at the same points.
     auto flush = [&](int64_t rt) {
-        if (issuer && ok && acc) mma_commit(bar_done);
-        if (ok && acc) ok = mbar_wait(bar_done, (uint32_t)(flushes & 1), A.flag);
+        drain();
         ok = __syncthreads_and(ok);
-        if (acc) ++flushes;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         uint32_t v[16];
         asm volatile(
@@ -257,8 +252,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             tile_row = rt;
         }
         // ---- x of this column group as the B operand (buffer u & 1), once
-        // every MMA that read the buffer (unit u - 2) has completed: the
-        // tile's slice t - 2 completes after them; then the CTA agrees
+        // every MMA that read the buffer (unit u - 2) has completed: each
+        // warp's slice t - 2 completes after them; then the CTA agrees
         uint8_t* B = s_B + (int)(u & 1) * kBBytes;
         if (t >= 2 && ok) ok = mbar_wait(&bar_buf[t & 1], (uint32_t)(((t >> 1) - 1) & 1), A.flag);
         ok = __syncthreads_and(ok);
@@ -302,8 +297,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             *reinterpret_cast<uint4*>(Ab + a_offset(trow, 0)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
             *reinterpret_cast<uint4*>(Ab + a_offset(trow, 1)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            // the tile's 128 rows are written and its threads agree that no wait gave up
-            ok = tile_sync_and(1 + tile, 128, ok);
+            // the warp's 32 rows are written (memory ordering among its lanes) and
+            // its lanes agree that no wait gave up
+            __syncwarp();
+            ok = __all_sync(0xffffffffu, ok);
             if (issuer && ok) {
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint64_t ad = smem_desc(smem_u32(Ab));
@@ -351,10 +348,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     }
     flush(tile_row);  // every thread leaves the unit loop at the same unit
 
-    // before the tensor memory is freed: the MMAs this tile committed are
+    // before the tensor memory is freed: the MMAs this warp committed are
     // done (bounded once more if a wait already gave up)
     if (t >= 1) mbar_wait(&bar_buf[(t - 1) & 1], (uint32_t)(((t - 1) >> 1) & 1), nullptr);
-    if (t >= 2) mbar_wait(&bar_buf[t & 1], (uint32_t)(((t >> 1) - 1) & 1), nullptr);
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == 0)
