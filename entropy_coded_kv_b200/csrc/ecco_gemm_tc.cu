@@ -26,10 +26,18 @@
 //     + 31, the lanes its own rows produced;
 //   - a warp writes a buffer again only after its own MMA that read it has
 //     completed.
-// x of the unit's column group is the B operand (double buffered by unit:
-// a CTA barrier per unit).  The centroids are read through the read-only
-// cache; shared memory holds the decode tables, the stream words, the decoded
-// symbols (for the records), A and B.
+// x of a unit's column group is its B operand, in a ring of 4 slots that all
+// threads fill two units ahead: a slot's "full" mbarrier completes when every
+// thread has written its share (and it is waited on before the unit's first
+// MMA); its "free" mbarrier completes when every warp's MMAs of the unit that
+// used it have finished and every warp has read its record corrections from
+// it (each warp's lane 0 commits to it after its last MMA of the unit, and
+// arrives on it after the records), and it is waited on before the slot is
+// refilled.  So no
+// barrier holds the warps together inside or between units: a warp can run up
+// to two units ahead of the slowest.  The centroids are read through the
+// read-only cache; shared memory holds the decode tables, the stream words,
+// the decoded symbols (for the records), A and the x ring.
 //
 // Outlier records are known only at the end of a block's stream, after its
 // slices went to the tensor cores, so their effect is added on CUDA cores as
@@ -38,12 +46,11 @@
 // atomics (a row tile is split over a few CTAs).
 //
 // Every wait on an mbarrier is bounded.  A wait that gives up counts itself
-// (ecco_device_timeouts) and raises a host-visible flag; the warp then issues
-// no more MMAs, the CTA agrees (a CTA-wide vote at the next unit and at every
-// accumulator read-out) to stop and to write nothing to y, waits once more
-// (bounded) for the MMAs it already committed, frees its tensor memory and
-// returns.  The next tensor-core ecco_decode_gemv call returns
-// ECCO_ERR_TIMEOUT.
+// (ecco_device_timeouts) and raises a host-visible flag; its warp then issues
+// no more MMAs and writes nothing more to y (the launch's y is incomplete and
+// the next tensor-core ecco_decode_gemv call returns ECCO_ERR_TIMEOUT); at the
+// end the CTA waits once more (bounded) for the MMAs it committed, frees its
+// tensor memory and returns.
 #include <mutex>
 
 #include "ecco_block.cuh"
@@ -67,9 +74,11 @@ constexpr size_t kOffWords = kOffLut + 65536;
 constexpr size_t kOffNib = kOffWords + (size_t)16 * kTcStride * 4;
 constexpr size_t kOffA = kOffNib + (size_t)16 * kTcThreads * 4;
 constexpr size_t kOffB = kOffA + (size_t)kTcTiles * 2 * kSliceBytes;
-constexpr size_t kOffBar = kOffB + (size_t)2 * kBBytes;
+constexpr int kBSlots = 4;                   // x ring: filled two units ahead
+constexpr size_t kOffBar = kOffB + (size_t)kBSlots * kBBytes;
 constexpr int kTcWarps = kTcThreads / 32;
-constexpr int kNumBars = 2 * kTcWarps;  // [warp][2]: the warp's MMAs on A buffer 0 / 1
+// [warp][2]: the warp's MMAs on A buffer 0 / 1; then x ring full[4], free[4]
+constexpr int kNumBars = 2 * kTcWarps + 2 * kBSlots;
 constexpr size_t kTcSmem = kOffBar + (size_t)kNumBars * 8 + 16 + kSmemAlign;
 constexpr uint32_t kTmemCols = 512;     // 24 warps x 16 fp32 columns, rounded up to a power of 2
 
@@ -183,8 +192,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     const int64_t u0 = A.units * blockIdx.x / gridDim.x, u1 = A.units * (blockIdx.x + 1) / gridDim.x;
 
     stage_lut<kTcThreads>(tb, s_lut, tid);
+    uint64_t* bar_full = &bars[2 * kTcWarps];
+    uint64_t* bar_free = &bars[2 * kTcWarps + kBSlots];
     if (tid == 0) {
-        for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2 * kTcWarps; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kBSlots; ++i) {
+            mbar_init(&bar_full[i], kTcThreads);  // every thread writes a share of x
+            // every warp twice: its lane 0 commits (the MMAs that read the slot are
+            // done) and arrives (its lanes have read their record corrections)
+            mbar_init(&bar_free[i], 2 * kTcWarps);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -208,22 +225,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     float corr[16];
 #pragma unroll
     for (int b = 0; b < 16; ++b) corr[b] = 0.0f;
-    bool ok = true;      // uniform in the warp after every slice, in the CTA after every unit start
+    bool ok = true;      // uniform in the warp after every slice
     int t = 0;           // slices so far (the A buffer is t & 1)
     bool acc = false;    // the warp's accumulators hold a partial sum
-    int64_t tile_row = (u0 < u1) ? u0 / A.gpr : 0;
+    const int64_t nu = u1 - u0;
+    int64_t tile_row = (nu > 0) ? u0 / A.gpr : 0;
 
+    // This thread's share of x for local unit l into its ring slot (l % 4),
+    // after the unit that used the slot before (l - 4) has no MMA left; then
+    // it announces the share on the slot's "full" mbarrier.
+    auto stage_x = [&](int64_t l) {
+        const int slot = (int)(l % kBSlots);
+        if (l >= kBSlots && ok) ok = mbar_wait(&bar_free[slot], (uint32_t)((l / kBSlots - 1) & 1), A.flag);
+        const int64_t g = (u0 + l) % A.gpr;
+        uint8_t* Bw = s_B + slot * kBBytes;
+        for (int e = tid; e < 16 * kG; e += kTcThreads) {
+            const int b = e & 15, k = e >> 4;
+            const uint16_t v = (b < A.batch) ? A.x[(int64_t)b * A.cols + g * kG + k] : (uint16_t)0;
+            *reinterpret_cast<uint16_t*>(Bw + (k >> 4) * kBSliceBytes + b_offset(b, k & 15)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // written by generic stores
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar_full[slot])) : "memory");
+    };
     // Waits until this warp's MMAs issued so far have completed (the commit of
     // the last slice completes after all of them).
     auto drain = [&]() {
         if (t >= 1 && ok) ok = mbar_wait(&bar_buf[(t - 1) & 1], (uint32_t)(((t - 1) >> 1) & 1), A.flag);
     };
     // Adds each thread's row of its warp's accumulators (plus the record
-    // corrections) to y and starts the next row tile from zero.  Called by
-    // every thread at the same points.
+    // corrections) to y and starts the next row tile from zero.  Per warp.
     auto flush = [&](int64_t rt) {
         drain();
-        ok = __syncthreads_and(ok);
+        ok = __all_sync(0xffffffffu, ok);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         uint32_t v[16];
         asm volatile(
@@ -245,30 +278,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     };
 
-    for (int64_t u = u0; u < u1; ++u) {
+    for (int64_t l = 0; l < 2 && l < nu; ++l) stage_x(l);
+
+    for (int64_t l = 0; l < nu; ++l) {
+        const int64_t u = u0 + l;
         const int64_t rt = u / A.gpr, g = u - rt * A.gpr;
         if (rt != tile_row) {
             flush(tile_row);
             tile_row = rt;
         }
-        // ---- x of this column group as the B operand (buffer u & 1), once
-        // every MMA that read the buffer (unit u - 2) has completed: each
-        // warp's slice t - 2 completes after them; then the CTA agrees
-        uint8_t* B = s_B + (int)(u & 1) * kBBytes;
-        if (t >= 2 && ok) ok = mbar_wait(&bar_buf[t & 1], (uint32_t)(((t >> 1) - 1) & 1), A.flag);
-        ok = __syncthreads_and(ok);
-        if (!ok) break;  // CTA-uniform
-        for (int e = tid; e < 16 * kG; e += kTcThreads) {
-            const int b = e & 15, k = e >> 4;
-            const uint16_t v = (b < A.batch) ? A.x[(int64_t)b * A.cols + g * kG + k] : (uint16_t)0;
-            *reinterpret_cast<uint16_t*>(B + (k >> 4) * kBSliceBytes + b_offset(b, k & 15)) = v;
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // B written by generic stores
-        __syncthreads();
+        if (l + 2 < nu) stage_x(l + 2);  // two units ahead
+        const int slot = (int)(l % kBSlots);
+        const uint8_t* B = s_B + slot * kBBytes;
 
-        // ---- this thread's row block
+        // ---- this thread's row block (and the next unit's on its way to L2)
         const int64_t row = rt * kTcThreads + tid;
         const bool row_ok = row < A.rows;
+        if (l + 1 < nu) {
+            const int64_t un = u + 1, rn = (un / A.gpr) * kTcThreads + tid;
+            if (rn < A.rows)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(A.blocks + (rn * A.gpr + (un % A.gpr)) * ECCO_BLOCK_BYTES));
+        }
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, q2 = q0, q3 = q0;
         if (row_ok) {
             const uint8_t* src = A.blocks + (row * A.gpr + g) * ECCO_BLOCK_BYTES;
@@ -293,6 +323,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
             nibs[(2 * sl + 1) * kTcThreads] = chunk_values(st, lkey, ws, kTcStride, vp, wb);
             const int buf = t & 1, use = t >> 1;
             if (use >= 1 && ok) ok = mbar_wait(&bar_buf[buf], (uint32_t)((use - 1) & 1), A.flag);
+            if (sl == 0 && ok) ok = mbar_wait(&bar_full[slot], (uint32_t)((l / kBSlots) & 1), A.flag);
             uint8_t* Ab = A0 + buf * kSliceBytes;
             *reinterpret_cast<uint4*>(Ab + a_offset(trow, 0)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
             *reinterpret_cast<uint4*>(Ab + a_offset(trow, 1)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
@@ -307,6 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 const uint64_t bd = smem_desc(smem_u32(B + sl * kBSliceBytes));
                 mma_bf16(tmem_d, ad, bd, acc ? 1u : 0u);
                 mma_commit(&bar_buf[buf]);
+                if (sl == 7) mma_commit(&bar_free[slot]);  // the x slot is free once these MMAs are done
             }
             acc = true;
         }
@@ -345,8 +377,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
                 }
             }
         }
+        __syncwarp();  // the warp's lanes are done with this unit's x slot
+        if (issuer)
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar_free[slot])) : "memory");
     }
-    flush(tile_row);  // every thread leaves the unit loop at the same unit
+    flush(tile_row);
 
     // before the tensor memory is freed: the MMAs this warp committed are
     // done (bounded once more if a wait already gave up)
