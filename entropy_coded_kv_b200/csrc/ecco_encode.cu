@@ -31,9 +31,12 @@
 // |x_m| / S_t is looked up by the bf16 magnitude of x_m, and s and 1/s by the
 // code, from tables the library builds on the device with the same IEEE
 // operations.  Thresholds, codeword lengths and codewords of one pattern share
-// one shared-memory row, so a symbol's position in the threshold search also
-// addresses its length and its codeword.  Every other fp32 operation is an
-// explicitly rounded intrinsic, so none is fused.
+// one shared-memory row, addressed by the symbol.  The threshold search costs
+// one comparison: the value's bucket in the pattern's map (two fused
+// multiply-adds, threshold_bucket) gives the number of thresholds in lower
+// buckets, and at most one threshold shares its bucket (patterns where two
+// do fall back to bisection).  Every other fp32 operation is an explicitly
+// rounded intrinsic, so none is fused.
 #include "ecco_internal.cuh"
 
 namespace ecco {
@@ -101,9 +104,28 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
     return v;
 }
 
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 // sym = number of thresholds T[0..13] of the row at shared address `R`
-// strictly below v (R9), by binary search: T[7] is in a register, the other
-// three levels read T[idx + 3], T[idx + 1], T[idx].
+// strictly below v (R9), by the bucket map: L = the pattern's 256 counts
+// (256-byte aligned), qm = its (a, b).  Thresholds in buckets below v's are
+// below v, those in buckets above are not, and the one threshold that may
+// share v's bucket is T[lo] (the thresholds are non-decreasing), so sym =
+// lo + (T[lo] < v); T[14] = +inf.
+__device__ __forceinline__ int quantise_bucket(uint32_t R, uint32_t L, float4 qm, float v)
+{
+    const uint32_t lo = lds_u8(L | threshold_bucket(v, qm.x, qm.y));
+    return (int)lo + ((__uint_as_float(lds_u32(R + 4u * lo)) < v) ? 1 : 0);
+}
+
+// The same count by bisection (patterns with two thresholds in one bucket):
+// T[7] is in a register, the other three levels read T[idx + 3], T[idx + 1],
+// T[idx].
 __device__ __forceinline__ int quantise(uint32_t R, float t7, float v)
 {
     int idx = (t7 < v) ? 8 : 0;
@@ -117,7 +139,7 @@ __device__ __forceinline__ int quantise(uint32_t R, float t7, float v)
 // within the group.  cent: centroids [64][16] (SEL = 1 only).
 template <int SEL, int G>
 __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, const uint32_t* rows,
-                                             const float* cent, uint32_t* buf, uint32_t* top,
+                                             uint32_t QL, const float4* qmap, const float* cent, uint32_t* buf, uint32_t* top,
                                              const float2 (&ends)[4], const uint16_t* src, uint8_t* dst, int hl,
                                              uint32_t gmask, int npat, Counters& cnt)
 {
@@ -216,10 +238,13 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
             const uint32_t Rq = (uint32_t)__cvta_generic_to_shared(rows) + (uint32_t)(q * kRow) * 4u;
             const float* Cq = cent + q * 16;
             const float tq = __uint_as_float(lds_u32(Rq + 28u));
+            const float4 qmq = qmap[q];
+            const uint32_t Lq = QL + (uint32_t)q * 256u;
             float d2[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float d = __fsub_rn(u[j], Cq[quantise(Rq, tq, u[j])]);
+                const int sj = (qmq.z == 0.0f) ? quantise_bucket(Rq, Lq, qmq, u[j]) : quantise(Rq, tq, u[j]);
+                const float d = __fsub_rn(u[j], Cq[sj]);
                 d2[j] = (owner && j == mj) ? 0.0f : __fmul_rn(d, d);
             }
             float v = __fadd_rn(__fadd_rn(__fadd_rn(d2[0], d2[1]), __fadd_rn(d2[2], d2[3])),
@@ -235,10 +260,17 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
 
     // ---- quantise (count of thresholds strictly below u); lengths
     const uint32_t R = (uint32_t)__cvta_generic_to_shared(rows) + (uint32_t)(p * kRow) * 4u;
-    const float t7 = __uint_as_float(lds_u32(R + 28u));
+    const float4 qm = qmap[p];
     int sym[8];
+    if (qm.z == 0.0f) {
+        const uint32_t L = QL + (uint32_t)p * 256u;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sym[j] = (j == jm) ? 15 : quantise(R, t7, u[j]);
+        for (int j = 0; j < 8; ++j) sym[j] = (j == jm) ? 15 : quantise_bucket(R, L, qm, u[j]);
+    } else {
+        const float t7 = __uint_as_float(lds_u32(R + 28u));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sym[j] = (j == jm) ? 15 : quantise(R, t7, u[j]);
+    }
     uint32_t acc = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc += lds_u32(R + 4u * (uint32_t)(kRowLens + sym[j]));
@@ -369,10 +401,13 @@ __global__ void __launch_bounds__(kEncWarps * 32, kEncCtasPerSm) encode_kernel(c
 {
     constexpr int kLanes = G / 8, kGpw = 32 / kLanes;  // lanes per group, groups per warp
     __shared__ uint32_t rows[kNPat * kRow];
+    __shared__ __align__(256) uint8_t qlo[kNPat * 256];  // bucket -> thresholds below, per pattern
+    __shared__ float4 qmap[kNPat];
     __shared__ float cent[SEL ? kNPat * 16 : 1];  // C[p][j] pattern-major (full-MSE selection)
     __shared__ uint32_t bufs[kGpw * kEncWarps][20];
     __shared__ uint32_t tops[kGpw * kEncWarps][kMaxRec];  // a group's outlier keys, in record order
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t QL = (uint32_t)__cvta_generic_to_shared(qlo);
     for (int i = tid; i < kGpw * kEncWarps * 20; i += blockDim.x) (&bufs[0][0])[i] = 0u;
     const int sub = lane / kLanes, hl = lane % kLanes;
     const uint32_t gmask = (uint32_t)((1ull << kLanes) - 1ull) << (kLanes * sub);
@@ -413,6 +448,15 @@ __global__ void __launch_bounds__(kEncWarps * 32, kEncCtasPerSm) encode_kernel(c
                 d[3] = v[k].w;
             }
         }
+        {
+            constexpr int kQVec = kNPat * 256 / 16, kPerQ = kQVec / (kEncWarps * 32);
+            uint4 w[kPerQ];
+#pragma unroll
+            for (int k = 0; k < kPerQ; ++k) w[k] = __ldg(reinterpret_cast<const uint4*>(&tb->qlo[0][0]) + tid + k * kEncWarps * 32);
+#pragma unroll
+            for (int k = 0; k < kPerQ; ++k) reinterpret_cast<uint4*>(qlo)[tid + k * kEncWarps * 32] = w[k];
+            if (tid < kNPat) qmap[tid] = __ldg(&tb->qmap[tid]);
+        }
         if constexpr (SEL == 1) {
             for (int i = tid; i < kNPat * 16; i += blockDim.x) cent[i] = tb->Ct[i & 15][i >> 4];
         }
@@ -430,7 +474,7 @@ __global__ void __launch_bounds__(kEncWarps * 32, kEncCtasPerSm) encode_kernel(c
         for (; item < end; item += kPerRound) {
             const uint16_t* src = S.src + (S.d.src_offset + r * S.d.src_row_stride + g) * G;
             uint8_t* dst = S.dst + (S.d.dst_offset + r * S.d.dst_row_stride + g) * ECCO_BLOCK_BYTES;
-            encode_group<SEL, G>(tb, rows, cent, buf, top, ends, src, dst, hl, gmask, P.npat, cnt);
+            encode_group<SEL, G>(tb, rows, QL, qmap, cent, buf, top, ends, src, dst, hl, gmask, P.npat, cnt);
             g += stride_g;
             r += stride_r;
             if (g >= gpr) {
@@ -459,10 +503,13 @@ cudaError_t run_encode(const EncParams<MAXSEG>& P, int select, cudaStream_t s)
     int64_t want = (P.total + per_cta - 1) / per_cta;
     int64_t cap = (int64_t)device_sm_count() * kEncCtasPerSm;  // one wave of resident CTAs
     int grid = (int)(want < cap ? want : cap);
-    if (select == ECCO_SELECT_MSE)
-        encode_kernel<MAXSEG, 1, G><<<grid, kEncWarps * 32, 0, s>>>(P);
-    else
-        encode_kernel<MAXSEG, 0, G><<<grid, kEncWarps * 32, 0, s>>>(P);
+    if constexpr (G == kG) {  // the full-MSE selection is offered for 128-value groups
+        if (select == ECCO_SELECT_MSE) {
+            encode_kernel<MAXSEG, 1, G><<<grid, kEncWarps * 32, 0, s>>>(P);
+            return cudaGetLastError();
+        }
+    }
+    encode_kernel<MAXSEG, 0, G><<<grid, kEncWarps * 32, 0, s>>>(P);
     return cudaGetLastError();
 }
 

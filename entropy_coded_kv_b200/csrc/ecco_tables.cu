@@ -130,6 +130,31 @@ __global__ void scale_tables_kernel(DevTables* t)
     }
 }
 
+// One thread per pattern: the map T[0] -> 0.01, T[13] -> 0.99 (before the
+// scaling by 255) and the per-bucket counts of thresholds below.  A pattern
+// whose map is not finite, or with two thresholds in one bucket, is marked
+// for bisection.
+__global__ void bucket_tables_kernel(DevTables* t)
+{
+    const int p = threadIdx.x;
+    if (p >= kNPat) return;
+    const float* T = t->T16[p];
+    const float a = __fdiv_rn(0.98f, __fsub_rn(T[kNCent - 2], T[0]));
+    const float b = __fsub_rn(0.01f, __fmul_rn(T[0], a));
+    bool dense = !(isfinite(a) && isfinite(b) && a > 0.0f);
+    uint32_t nb[kNCent - 1];
+    for (int k = 0; k < kNCent - 1; ++k) {
+        nb[k] = threshold_bucket(T[k], a, b);
+        if (k && nb[k] <= nb[k - 1]) dense = true;
+    }
+    for (uint32_t n = 0; n < 256; ++n) {
+        uint32_t lo = 0;
+        for (int k = 0; k < kNCent - 1; ++k) lo += (nb[k] < n) ? 1u : 0u;
+        t->qlo[p][n] = (uint8_t)lo;
+    }
+    t->qmap[p] = make_float4(a, b, dense ? 1.0f : 0.0f, 0.0f);
+}
+
 }  // namespace
 
 extern "C" int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables** out)
@@ -160,6 +185,7 @@ extern "C" int ecco_tables_create(const void* blob, size_t nbytes, ecco_tables**
     delete host;
     if (e == cudaSuccess) {
         scale_tables_kernel<<<32768 / 256, 256>>>(d);
+        bucket_tables_kernel<<<1, kNPat>>>(d);
         e = cudaGetLastError();
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
     }

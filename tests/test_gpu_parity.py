@@ -40,6 +40,18 @@ def table_set(name: str) -> bytes:
             seed = int(name[6:])
             st = {0: 0.02 * 4 / 448, 1: None, 2: 2.0 ** -40, 3: 1.0}.get(seed)
             _TABLE_CACHE[name] = W.random_tables(seed, S_t=st)
+        elif name == "crowded":
+            # every other pattern with 8 centroids 1e-5 apart: several of its
+            # thresholds share one bucket of the encoder's threshold map, so
+            # those patterns take the bisection search
+            blob = W.random_tables(11)
+            S_t = float(np.frombuffer(blob, np.float32, 1, 8)[0])
+            C = np.frombuffer(blob, np.float32, 64 * 15, 16).reshape(64, 15).copy()
+            lens = np.frombuffer(blob, np.uint8, 64 * 4 * 16, 16 + 64 * 15 * 4).reshape(64, 4, 16)
+            for p in range(0, 64, 2):
+                C[p, 3:11] = C[p, 3] + np.arange(8, dtype=np.float32) * np.float32(1e-5)
+            assert np.all(np.diff(C, axis=1) > 0)
+            _TABLE_CACHE[name] = W.pack_tables(S_t, C, lens)
         elif name == "learned_c1":
             _TABLE_CACHE[name] = learn_tables(W.c1_matrix(), seed=0)
         elif name == "learned_kv":
@@ -83,7 +95,7 @@ def inputs(kind: str, n_groups: int, seed: int) -> np.ndarray:
     return bits(x.to(torch.bfloat16))
 
 
-TABLES = ["random0", "random1", "random2", "random3", "learned_c1", "learned_kv", "learned_w"]
+TABLES = ["random0", "random1", "random2", "random3", "crowded", "learned_c1", "learned_kv", "learned_w"]
 KINDS = ["gauss", "t5", "kv", "c1", "special"]
 
 
