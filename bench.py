@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--workload", default="longctx", choices=["kv", "c1", "mlp", "model", "longctx", "attn", "select", "act"])
     ap.add_argument("--attention", default="staged", choices=["staged", "fused"],
                     help="attn workload: decode_attention_staged (default) or the single fused kernel")
+    ap.add_argument("--decoder", default="serial", choices=["serial", "speculative"],
+                    help="kv workload: decode with the thread-per-block walk (default) or the warp-parallel "
+                         "speculative decoder (ecco_decode_speculative, one launch per tensor)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
@@ -231,6 +234,7 @@ class KVWorkload(Workload):
     desc = ("Llama-3-8B-shaped one-layer KV cache, K and V each [8, 8, 4096, 128] bf16: "
             "encode the last 64 tokens (8,192 groups) + decode the full cache (524,288 blocks)")
     B, H, S, D, T = 8, 8, 4096, 128, 64
+    speculative = False  # decode through ecco_decode_speculative instead
 
     def __init__(self, dev, seed_offset=0):
         import torch
@@ -253,8 +257,17 @@ class KVWorkload(Workload):
         self.append = ecco.kv_append_desc(self.rows, self.T, self.S, self.S - self.T)
         self.app = [ecco.Seg(self.tables[i], self.new[i], self.blocks[i], self.append) for i in range(2)]
         self.dec = [ecco.Seg(self.tables[i], self.blocks[i], self.out[i]) for i in range(2)]
-        self.launches_per_step = 2
+        self.launches_per_step = 3 if self.speculative else 2
+        if self.speculative:
+            self.desc = self.desc + "; decode by the warp-parallel speculative decoder (one launch per tensor)"
         self.dec_ms = []
+
+    def _decode(self):
+        if self.speculative:
+            for i in range(2):
+                self.ecco.decode(self.blocks[i], self.tables[i], out=self.out[i], speculative=True)
+        else:
+            self.ecco.decode_multi(self.dec)
 
     def bytes_decoded(self):
         return 2 * self.n * 256
@@ -269,7 +282,7 @@ class KVWorkload(Workload):
         if record:
             a, b = _events(self.torch)
             a.record()
-        e.decode_multi(self.dec)
+        self._decode()
         if record:
             b.record()
             self.dec_ms.append((a, b))
@@ -278,7 +291,7 @@ class KVWorkload(Workload):
         """(kernel name, algorithmic bytes per launch, launch ms list)."""
         self.torch.cuda.synchronize()
         ms = [a.elapsed_time(b) for a, b in self.dec_ms]
-        return "decode_kernel", 2 * self.n * (64 + 256), ms
+        return ("decode_spec_kernel" if self.speculative else "decode_kernel"), 2 * self.n * (64 + 256), ms
 
     # ---- end to end through the public API with host buffers
     def e2e_setup(self):
@@ -297,7 +310,7 @@ class KVWorkload(Workload):
             self.d_new[i].copy_(self.h_new[i], non_blocking=True)
             self.blocks[i].copy_(self.h_blocks[i], non_blocking=True)
         e.encode_multi(self.e2e_app)
-        e.decode_multi(self.dec)
+        self._decode()
         for i in range(2):
             self.h_out[i].copy_(self.out[i], non_blocking=True)
 
@@ -1129,6 +1142,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     AttnWorkload.path = args.attention
+    KVWorkload.speculative = args.decoder == "speculative"
     ModelWorkload.layers = LongCtxWorkload.layers = args.layers
     wl = WORKLOADS[args.workload](dev, seed_offset=0)
     if getattr(wl, "layers", 32) != 32:
@@ -1233,6 +1247,7 @@ def main():
 # profiles/traffic.json is used only while these files are unchanged.
 KERNEL_SOURCES = {
     "decode_kernel": ["ecco_decode.cu", "ecco_block.cuh"],
+    "decode_spec_kernel": ["ecco_decode_spec.cu", "ecco_block.cuh"],
     "decode_kernel<G=64>": ["ecco_decode.cu", "ecco_block.cuh"],
     "encode_kernel<.,SEL=1>": ["ecco_encode.cu", "ecco_internal.cuh"],
     "decode_kernel+attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_decode.cu", "ecco_block.cuh"],

@@ -130,8 +130,9 @@ def encode(x: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
 
 
 def decode(blocks: torch.Tensor, tables: Tables, out: torch.Tensor | None = None,
-           desc: Desc | None = None) -> torch.Tensor:
-    """uint8 blocks [n, 64] -> bf16 [n, 128]."""
+           desc: Desc | None = None, speculative: bool = False) -> torch.Tensor:
+    """uint8 blocks [n, 64] -> bf16 [n, 128].  speculative=True runs the
+    warp-parallel decoder (ecco_decode_speculative): same output."""
     _check_tensor(blocks, torch.uint8, "blocks", tables.device)
     n_blocks = blocks.numel() // BLOCK_BYTES
     if desc is None:
@@ -140,9 +141,10 @@ def decode(blocks: torch.Tensor, tables: Tables, out: torch.Tensor | None = None
         out = torch.empty((desc.rows * desc.groups_per_row, GROUP), dtype=torch.bfloat16, device=blocks.device)
     _check_tensor(out, torch.bfloat16, "out", tables.device)
     _bounds(desc, n_blocks, out.numel() // GROUP)
-    rc = _lib.load().ecco_decode(tables.handle, ctypes.c_void_p(blocks.data_ptr()), desc,
-                                 ctypes.c_void_p(out.data_ptr()), _stream(blocks.device))
-    _lib.check(rc, "ecco_decode")
+    fn = "ecco_decode_speculative" if speculative else "ecco_decode"
+    rc = getattr(_lib.load(), fn)(tables.handle, ctypes.c_void_p(blocks.data_ptr()), desc,
+                                  ctypes.c_void_p(out.data_ptr()), _stream(blocks.device))
+    _lib.check(rc, fn)
     return out
 
 

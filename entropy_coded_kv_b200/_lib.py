@@ -24,7 +24,7 @@ TABLES_BYTES = 7952
 MAX_SEGMENTS = 256
 
 EXPORTED = [
-    "ecco_tables_create", "ecco_tables_destroy", "ecco_select_encode", "ecco_decode",
+    "ecco_tables_create", "ecco_tables_destroy", "ecco_select_encode", "ecco_decode", "ecco_decode_speculative",
     "ecco_decode_gemv", "ecco_decode_multi", "ecco_encode_multi", "ecco_strerror",
     "ecco_abi_version", "ecco_device_timeouts", "ecco_decode_attention",
     "ecco_decode_attention_workspace_bytes", "ecco_decode_attention_static", "ecco_select_encode_ex",
@@ -69,6 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ecco_tables_destroy.argtypes = [P]
     L.ecco_select_encode.argtypes = [P, P, Desc, P, P, P]
     L.ecco_decode.argtypes = [P, P, Desc, P, P]
+    L.ecco_decode_speculative.argtypes = [P, P, Desc, P, P]
     L.ecco_select_encode_ex.argtypes = [P, P, Desc, P, P, I, I, P]
     L.ecco_select_encode_act.argtypes = [P, P, Desc, P, P, P]
     L.ecco_learn_tables.argtypes = [P, I64, I, I, ctypes.c_uint64, P, ctypes.c_size_t, P]

@@ -124,6 +124,18 @@ extern "C" int ecco_decode(const ecco_tables* t, const uint8_t* blocks, ecco_des
     return status(launch_decode(t, blocks, d, y, (cudaStream_t)stream));
 }
 
+extern "C" int ecco_decode_speculative(const ecco_tables* t, const uint8_t* blocks, ecco_desc d, uint16_t* y,
+                                       void* stream)
+{
+    int rc = check_tables(t);
+    if (rc) return rc;
+    if ((rc = check_desc(d))) return rc;
+    if (d.rows == 0 || d.groups_per_row == 0) return ECCO_OK;
+    if (!blocks || !y) return ECCO_ERR_ARG;
+    if (!aligned16(blocks) || !aligned16(y)) return ECCO_ERR_ALIGN;
+    return status(launch_decode_spec(t, blocks, d, y, (cudaStream_t)stream));
+}
+
 extern "C" int ecco_decode_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows,
                                 int64_t cols, const uint16_t* x, int batch, float* y, void* stream)
 {

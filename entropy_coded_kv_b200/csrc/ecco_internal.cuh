@@ -76,6 +76,8 @@ cudaError_t launch_encode(const ecco_tables* t, const uint16_t* x, const ecco_de
                           int select = ECCO_SELECT_MINMAX, int npat = kNPat);
 cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
                           uint16_t* y, cudaStream_t s);
+cudaError_t launch_decode_spec(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
+                               uint16_t* y, cudaStream_t s);
 cudaError_t launch_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,
                         const uint16_t* x, int batch, float* y, cudaStream_t s);
 cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t rows, int64_t cols,

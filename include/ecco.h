@@ -165,6 +165,19 @@ int ecco_decode_act(const ecco_tables* tables, const uint8_t* blocks, ecco_desc 
 int ecco_decode(const ecco_tables* tables, const uint8_t* blocks, ecco_desc desc,
                 uint16_t* y_bf16, void* stream);
 
+/* The same decoder organised as the review page's parallel decompressor
+ * (Fig. 8 caption; referee major comment 1: sub-decoders start on
+ * overlapping segments at every candidate bit offset and a tree merge picks
+ * the true chain): one warp per block, each lane decodes at every bit
+ * position of a 16-bit payload segment, the lanes' offset maps are composed
+ * by a shuffle scan, and each lane emits the codewords of its segment.  The
+ * output is bit-identical to ecco_decode's; arguments, alignment and errors
+ * are ecco_decode's.  It does several times the work per block of the
+ * one-thread-per-block walk and is slower on this hardware; it is offered
+ * for comparison. */
+int ecco_decode_speculative(const ecco_tables* tables, const uint8_t* blocks, ecco_desc desc,
+                            uint16_t* y_bf16, void* stream);
+
 /* Fused decode + matrix-vector product ("Normalized memory requests for a
  * GEMM kernel", review page figure list): y[b][r] = sum_k W~[r][k] x[b][k],
  * on CUDA cores for batch 1..4 and on the tcgen05 tensor cores for 5..16,
