@@ -1249,7 +1249,7 @@ KERNEL_SOURCES = {
     "decode_kernel": ["ecco_decode.cu", "ecco_block.cuh"],
     "decode_spec_kernel": ["ecco_decode_spec.cu", "ecco_block.cuh"],
     "decode_kernel<G=64>": ["ecco_decode.cu", "ecco_block.cuh"],
-    "encode_kernel<.,SEL=1>": ["ecco_encode.cu", "ecco_internal.cuh"],
+    "encode_kernel<.,SEL=1>": ["ecco_encode.cu", "ecco_bucket.cuh"],
     "decode_kernel+attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_decode.cu", "ecco_block.cuh"],
     "attn_split_kernel+attn_merge_kernel": ["ecco_attention.cu", "ecco_block.cuh"],
 }

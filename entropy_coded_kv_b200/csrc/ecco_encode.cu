@@ -37,6 +37,7 @@
 // buckets, and at most one threshold shares its bucket (patterns where two
 // do fall back to bisection).  Every other fp32 operation is an explicitly
 // rounded intrinsic, so none is fused.
+#include "ecco_bucket.cuh"
 #include "ecco_internal.cuh"
 
 namespace ecco {

@@ -14,6 +14,7 @@
 #include <cstring>
 #include <new>
 
+#include "ecco_bucket.cuh"
 #include "ecco_internal.cuh"
 
 namespace {
