@@ -44,7 +44,17 @@ constexpr size_t dec_smem()
            (G == kG ? 0 : (size_t)dec_threads<G>() * kRowWords * 4);
 }
 
-// WIDE: 32-byte stores (output 32-byte aligned), else 16-byte stores.
+// 32 bytes from global memory through the read-only path (one 256-bit load).
+__device__ __forceinline__ void ldg_nc_v8(const void* p, uint4& a, uint4& b)
+{
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
+// WIDE: blocks and output both 32-byte aligned: 32-byte block loads and
+// stores (a 64-byte block in two loads: 2.7% faster on the long-context
+// cache than four 16-byte loads); else 16-byte loads and stores.
 template <bool WIDE>
 __device__ __forceinline__ void store16(uint16_t* dst, const uint32_t a[4], const uint32_t b[4])
 {
@@ -131,8 +141,16 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(S.src + (S.d.src_offset + r * S.d.src_row_stride + g) *
                                                                             ECCO_BLOCK_BYTES));
 
-            uint4 q0 = ldg_nc_v4(src), q1 = ldg_nc_v4(src + 16), q2 = ldg_nc_v4(src + 32),
-                  q3 = ldg_nc_v4(src + 48);
+            uint4 q0, q1, q2, q3;
+            if constexpr (WIDE) {
+                ldg_nc_v8(src, q0, q1);
+                ldg_nc_v8(src + 32, q2, q3);
+            } else {
+                q0 = ldg_nc_v4(src);
+                q1 = ldg_nc_v4(src + 16);
+                q2 = ldg_nc_v4(src + 32);
+                q3 = ldg_nc_v4(src + 48);
+            }
             const uint32_t code = q0.x & 0xffu;
             if (scale_code_is_null(code)) {
                 const uint32_t z[4] = {0u, 0u, 0u, 0u};
@@ -218,7 +236,7 @@ cudaError_t launch_decode(const ecco_tables* t, const uint8_t* blocks, const ecc
     P.n_seg = 1;
     P.total = d.rows * d.groups_per_row;
     P.seg[0] = DecSeg{t->d, blocks, y, d, 0, P.total};
-    return wide_ok(y) ? run_decode<true, 1>(P, s) : run_decode<false, 1>(P, s);
+    return (wide_ok(y) && wide_ok(blocks)) ? run_decode<true, 1>(P, s) : run_decode<false, 1>(P, s);
 }
 
 cudaError_t launch_decode_act(const ecco_tables* t, const uint8_t* blocks, const ecco_desc& d,
@@ -228,7 +246,7 @@ cudaError_t launch_decode_act(const ecco_tables* t, const uint8_t* blocks, const
     P.n_seg = 1;
     P.total = d.rows * d.groups_per_row;
     P.seg[0] = DecSeg{t->d, blocks, y, d, 0, P.total};
-    return wide_ok(y) ? run_decode<true, 1, kGAct>(P, s) : run_decode<false, 1, kGAct>(P, s);
+    return (wide_ok(y) && wide_ok(blocks)) ? run_decode<true, 1, kGAct>(P, s) : run_decode<false, 1, kGAct>(P, s);
 }
 
 // Segments are packed into launches of at most kMultiSeg; empty ones are skipped.
@@ -248,7 +266,7 @@ cudaError_t launch_decode_multi(const ecco_segment* segs, int n, cudaStream_t s)
                 P.seg[P.n_seg++] = DecSeg{segs[i].tables->d, static_cast<const uint8_t*>(segs[i].src),
                                           static_cast<uint16_t*>(segs[i].dst), d, P.total, cnt};
                 P.total += cnt;
-                wide = wide && wide_ok(segs[i].dst);
+                wide = wide && wide_ok(segs[i].dst) && wide_ok(segs[i].src);
             }
             ++i;
         }

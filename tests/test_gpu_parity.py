@@ -174,6 +174,24 @@ def test_decode_into_16_byte_aligned_output():
     assert (bits(flat[:8]) == 0).all()
 
 
+def test_decode_from_16_byte_aligned_blocks():
+    """Blocks aligned to 16 but not 32 bytes take the 16-byte-load variant."""
+    blob = table_set("learned_kv")
+    xb = inputs("kv", 700, seed=5)
+    blocks, _ = oracle.encode(blob, xb, nthreads=8)
+    t = ecco.Tables(blob, DEV)
+    flat = torch.zeros(700 * 64 + 16, dtype=torch.uint8, device=DEV)
+    blk = flat[16:].view(700, 64)
+    blk.copy_(torch.from_numpy(blocks).to(DEV))
+    assert blk.data_ptr() % 32 == 16
+    for dec in (ecco.decode, lambda b, tt: ecco.decode(b, tt, speculative=True)):
+        y = dec(blk, t)
+        np.testing.assert_array_equal(bits(y).reshape(-1, 128), oracle.decode(blob, blocks, nthreads=8))
+    y = torch.empty((700, 128), dtype=torch.bfloat16, device=DEV)
+    ecco.decode_multi([ecco.Seg(t, blk, y)])
+    np.testing.assert_array_equal(bits(y).reshape(-1, 128), oracle.decode(blob, blocks, nthreads=8))
+
+
 def test_empty_inputs_enqueue_nothing():
     t = ecco.Tables(table_set("random0"), DEV)
     x = torch.empty(0, dtype=torch.bfloat16, device=DEV)
