@@ -5,18 +5,20 @@
 // memory (the review page's figure list: "Normalized Memory Requests for a
 // GEMM Kernel" -- compressed weights are what crosses the memory bus).
 //
-// Layout of the work: a unit is one row per thread (1024 rows at batch 1, 512
-// at batch 2..4) x one column group; a CTA owns a balanced, contiguous range of units in (row tile, column
-// group) order and stays resident (one CTA per SM), so every SM gets the same
-// amount of work instead of a grid of whole tiles that leaves part of the last
-// wave idle.  A warp owns 32 consecutive rows, so at every step all lanes need
-// the same x[k] (a broadcast shared-memory read); x is staged in windows of 32
-// column groups.  Each lane decodes its row's block serially (one lookup per
-// symbol, as in the decoder) and multiplies every decoded bf16 value, exactly,
-// in fp32 against the batch of x.  An outlier record replaces the value of its
-// element, so its contribution is corrected by (new - old) * x, with the old
-// symbol kept in shared memory.  A thread's row sum is added to y (fp32
-// atomics) when its unit range moves to the next row tile and at the end.
+// Layout of the work: an item is one strip of 32 rows (a warp, a lane per
+// row) x one column group, numbered column group by column group.  Each CTA
+// (one per SM, resident) owns a balanced, contiguous range of items and runs
+// it in rounds of one item per warp, so CTAs differ by at most one item and
+// a CTA's last round is short (whole units of one row per thread would leave
+// the SMs that own one unit fewer idle for a quarter of the launch at the
+// 14336 x 4096 shape).  All lanes of a warp need the same x[k] at every step
+// (a broadcast shared-memory read); x is staged in windows of 32 column
+// groups, restaged when a round reaches past the window.  Each lane decodes
+// its row's block serially (one lookup per symbol, as in the decoder) and
+// multiplies every decoded bf16 value, exactly, in fp32 against the batch of
+// x.  An outlier record replaces the value of its element, so its
+// contribution is corrected by (new - old) * x, with the old symbol kept in
+// shared memory.  Each item's row sums are added to y with fp32 atomics.
 #include "ecco_block.cuh"
 
 namespace ecco {
@@ -58,45 +60,39 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
 
     stage_tables<kGvThreads>(tb, s_lut, s_Ct, tid);
     const float S_t = tb->S_t;
-    const int64_t tiles = (rows + kGvThreads - 1) / kGvThreads;
-    const int64_t units = tiles * gpr;
-    const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
+    constexpr int kWarps = kGvThreads / 32;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int64_t strips = (rows + 31) / 32;
+    const int64_t items = strips * gpr;  // item q: column group q / strips, strip q % strips
+    const int64_t qa = items * blockIdx.x / gridDim.x, qb = items * (blockIdx.x + 1) / gridDim.x;
 
     uint32_t* ws = s_w + tid;
     uint32_t* nibs = s_nib + tid;
-    float acc[B];
-#pragma unroll
-    for (int bb = 0; bb < B; ++bb) acc[bb] = 0.0f;
-    int64_t cur_tile = u0 / gpr, cur_win = -1;
+    int64_t win0 = -1;  // first column group of the staged x window
 
-    for (int64_t u = u0; u < u1; ++u) {
-        const int64_t tile = u / gpr, gcol = u - tile * gpr;
-        if (tile != cur_tile) {  // this thread's row changes: add its sum to y
-            const int64_t prow = cur_tile * kGvThreads + tid;
-            if (prow < rows) {
-#pragma unroll
-                for (int bb = 0; bb < B; ++bb)
-                    if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + prow], acc[bb]);
-            }
-#pragma unroll
-            for (int bb = 0; bb < B; ++bb) acc[bb] = 0.0f;
-            cur_tile = tile;
-        }
-        const int64_t win = gcol / kGvWin;
-        if (win != cur_win) {  // uniform across the CTA
-            __syncthreads();   // the previous window is no longer read (and the tables are staged)
-            const int64_t k0 = win * kGvWin * kG;
+    for (int64_t q0 = qa; q0 < qb; q0 += kWarps) {
+        // the round's column groups must lie in the window (uniform across the CTA)
+        const int64_t g_first = q0 / strips, g_last = (min(q0 + kWarps, qb) - 1) / strips;
+        if (win0 < 0 || g_first < win0 || g_last >= win0 + kGvWin) {
+            __syncthreads();  // the previous window is no longer read (and the tables are staged)
+            win0 = g_first;
+            const int64_t k0 = win0 * kG;
             const int nk = (int)min((int64_t)kGvWin * kG, cols - k0);
             for (int i = tid; i < kGvWin * kG * B; i += kGvThreads) {
                 const int k = i / B, bb = i - k * B;
                 s_x[i] = (bb < batch && k < nk) ? bf16_bits_to_f32(x[(int64_t)bb * cols + k0 + k]) : 0.0f;
             }
             __syncthreads();
-            cur_win = win;
         }
-        const int64_t row = tile * kGvThreads + tid;
+        const int64_t q = q0 + warp;
+        if (q >= qb) continue;  // this warp has no item in the CTA's short last round
+        const int64_t gcol = q / strips;
+        const int64_t row = (q - gcol * strips) * 32 + lane;
         const bool row_ok = row < rows;
-        const float* xs = s_x + (gcol - win * kGvWin) * kG * B;
+        const float* xs = s_x + (gcol - win0) * kG * B;
+        float acc[B];
+#pragma unroll
+        for (int bb = 0; bb < B; ++bb) acc[bb] = 0.0f;
         {
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, q2 = q0, q3 = q0;
         if (row_ok) {
@@ -152,8 +148,7 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
                 seen2 |= (q == 2u) ? bit : 0u;
                 seen3 |= (q == 3u) ? bit : 0u;
                 if (was) continue;
-                float nv = bf16_bits_to_f32(
-                    f32_to_bf16_bits(__fmul_rn(s, __fdiv_rn((float)(int)(int8_t)(uint8_t)(rec >> 7), 127.0f))));
+                float nv = bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(s, q_over_127((int)(int8_t)(uint8_t)(rec >> 7)))));
                 uint32_t osym = (nibs[(i >> 3) * kGvThreads] >> (4 * (i & 7))) & 15u;
                 uint32_t ow = (osym < 8) ? ((osym < 4) ? vp.lo[0] : vp.lo[1]) : ((osym < 12) ? vp.lo[2] : vp.lo[3]);
                 uint32_t oh = (osym < 8) ? ((osym < 4) ? vp.hi[0] : vp.hi[1]) : ((osym < 12) ? vp.hi[2] : vp.hi[3]);
@@ -166,12 +161,11 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
             }
         }
         }
-    }
-    const int64_t prow = cur_tile * kGvThreads + tid;
-    if (u1 > u0 && prow < rows) {
+        if (row_ok) {
 #pragma unroll
-        for (int bb = 0; bb < B; ++bb)
-            if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + prow], acc[bb]);
+            for (int bb = 0; bb < B; ++bb)
+                if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + row], acc[bb]);
+        }
     }
 }
 
@@ -185,8 +179,10 @@ cudaError_t run_gemv(const ecco_tables* t, const uint8_t* blocks, int64_t rows, 
     cudaError_t e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)batch * (size_t)rows, s);
     if (e != cudaSuccess) return e;
     const int64_t gpr = cols / kG;
-    const int64_t units = (rows + gv_threads<B>() - 1) / gv_threads<B>() * gpr;
-    const int grid = (int)(units < device_sm_count() ? units : device_sm_count());  // one resident CTA per SM
+    const int64_t items = (rows + 31) / 32 * gpr;  // 32-row strips x column groups
+    const int64_t per_cta = gv_threads<B>() / 32;   // one item per warp per round
+    const int64_t want = (items + per_cta - 1) / per_cta;
+    const int grid = (int)(want < device_sm_count() ? want : device_sm_count());  // one resident CTA per SM
     gemv_kernel<B><<<grid, gv_threads<B>(), gv_smem<B>(), s>>>(t->d, blocks, rows, gpr, x, batch, cols, y);
     return cudaGetLastError();
 }

@@ -262,7 +262,7 @@ def gemv_check(blob, blocks_np, rows, cols, xb, y):
 
 
 @pytest.mark.parametrize("batch", [1, 2, 3, 4, 5, 16])
-@pytest.mark.parametrize("rows,cols", [(700, 384), (64, 1024), (1030, 512)])
+@pytest.mark.parametrize("rows,cols", [(700, 384), (64, 1024), (1030, 512), (5, 8192), (33, 4224)])
 def test_gemv_within_tolerance(batch, rows, cols):
     blob = table_set("learned_w")
     wb = inputs("t5", rows * cols // 128, seed=rows + cols)
