@@ -21,6 +21,8 @@
 // output values bf16(s * C[p][j]) as register byte planes, decode the stream
 // 8 symbols at a time (ecco_block.cuh), write each 16 decoded values with one
 // 32-byte store, then apply the outlier records of an unclipped stream.
+#include <algorithm>
+
 #include "ecco_block.cuh"
 
 namespace ecco {
@@ -216,9 +218,12 @@ cudaError_t run_decode(const DecParams<MAXSEG>& P, cudaStream_t s)
     static std::atomic<uint64_t> configured{0};
     cudaError_t e = set_max_smem_once(configured, (const void*)decode_kernel<WIDE, MAXSEG, G>, dec_smem<G>());
     if (e != cudaSuccess) return e;
-    int64_t want = (P.total + dec_threads<G>() - 1) / dec_threads<G>();
-    int64_t cap = device_sm_count();
-    int grid = (int)(want < cap ? want : cap);
+    // one resident CTA per SM; a small launch is spread over the SMs (at
+    // least 16 blocks per CTA) rather than filling a few of them, since each
+    // thread walks its blocks serially: 2,048 blocks run on 128 SMs, not 2
+    const int64_t cap = device_sm_count();
+    const int64_t want = std::max((P.total + dec_threads<G>() - 1) / dec_threads<G>(), (P.total + 15) / 16);
+    const int grid = (int)(want < cap ? want : cap);
     decode_kernel<WIDE, MAXSEG, G><<<grid, dec_threads<G>(), dec_smem<G>(), s>>>(P);
     return cudaGetLastError();
 }
