@@ -45,6 +45,9 @@ int check_desc(const ecco_desc& d)
     const int64_t lim = (int64_t)1 << 40;
     if (d.rows > lim || d.groups_per_row > lim) return ECCO_ERR_ARG;
     if (d.rows > 0 && d.groups_per_row > 0) {
+        // at most 2^31 - 2048 groups per tensor and call (512 GiB of bf16):
+        // the kernels index a tensor's groups with 32-bit integers
+        if (d.rows > (((int64_t)1 << 31) - 2048) / d.groups_per_row) return ECCO_ERR_ARG;
         if (d.src_row_stride > lim / (d.rows > 1 ? d.rows : 1)) return ECCO_ERR_ARG;
         if (d.dst_row_stride > lim / (d.rows > 1 ? d.rows : 1)) return ECCO_ERR_ARG;
         if (d.src_offset > lim || d.dst_offset > lim) return ECCO_ERR_ARG;

@@ -84,7 +84,10 @@ typedef struct ecco_tables ecco_tables;
  * the last T tokens of a [B, H, S, 128] KV cache from a [B, H, T, 128] tensor:
  * rows = B*H, groups_per_row = T, src_row_stride = T, dst_row_stride = S,
  * src_offset = 0, dst_offset = S - T.  All fields >= 0; when rows > 1,
- * dst_row_stride >= groups_per_row (destination rows may not overlap). */
+ * dst_row_stride >= groups_per_row (destination rows may not overlap);
+ * rows * groups_per_row <= 2^31 - 2048 (512 GiB of bf16 per tensor and call:
+ * the kernels index a tensor's groups with 32-bit integers); other entries
+ * return ECCO_ERR_ARG. */
 typedef struct {
     int64_t rows;
     int64_t groups_per_row;

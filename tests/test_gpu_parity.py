@@ -244,6 +244,13 @@ def test_argument_errors_return_codes_and_launch_nothing():
     neg = _lib.Desc(1, -4, 4, 4, 0, 0)
     assert lib.ecco_decode(t.handle, ctypes.c_void_p(out.data_ptr()), neg, ctypes.c_void_p(x.data_ptr()),
                            None) == _lib.ECCO_ERR_ARG
+    # more than 2^31 - 2048 groups in one call (the kernels' 32-bit group index)
+    huge = _lib.Desc(1 << 20, 1 << 11, 1 << 11, 1 << 11, 0, 0)
+    for fn in (lib.ecco_decode, lib.ecco_decode_speculative):
+        assert fn(t.handle, ctypes.c_void_p(out.data_ptr()), huge, ctypes.c_void_p(x.data_ptr()),
+                  None) == _lib.ECCO_ERR_ARG
+    assert lib.ecco_select_encode(t.handle, ctypes.c_void_p(x.data_ptr()), huge, ctypes.c_void_p(out.data_ptr()),
+                                  None, None) == _lib.ECCO_ERR_ARG
     assert lib.ecco_decode_gemv(t.handle, ctypes.c_void_p(out.data_ptr()), 1, 100, ctypes.c_void_p(x.data_ptr()),
                                 1, ctypes.c_void_p(x.data_ptr()), None) == _lib.ECCO_ERR_ARG
     assert lib.ecco_decode_gemv(t.handle, ctypes.c_void_p(out.data_ptr()), 1, 128, ctypes.c_void_p(x.data_ptr()),
