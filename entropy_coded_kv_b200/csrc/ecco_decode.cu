@@ -229,12 +229,36 @@ __global__ void __launch_bounds__(dec_threads<G>(), 1) decode_kernel(const __gri
                 }
             }
             if constexpr (kRows) {
+                // A warp whose 32 rows follow one another in the output (every
+                // lane here, each row right after the previous lane's) writes
+                // them as G/16 fully contiguous 1 KB stores: lane L stores bytes
+                // 32 L .. 32 L + 31 of each, read from the staged row they
+                // belong to, so an instruction touches 8 rows instead of 32.
+                const unsigned am = __activemask();
+                const int lane = tid & 31;
+                const uintptr_t d0 = __shfl_sync(am, reinterpret_cast<uintptr_t>(dst), 0);
+                const bool follows = reinterpret_cast<uintptr_t>(dst) == d0 + (uintptr_t)lane * G * 2;
+                if (am == 0xffffffffu && __all_sync(am, follows)) {
+                    __syncwarp();  // every lane's row, records included, is staged
+                    const uint32_t* wrows = s_w + 16 * kWordStride + (tid & ~31) * kRowWords;
 #pragma unroll
-                for (int c = 0; c < G / 16; ++c) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(row + 8 * c);
-                    const uint4 b = *reinterpret_cast<const uint4*>(row + 8 * c + 4);
-                    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-                    store16<WIDE>(dst + 16 * c, wa, wb);
+                    for (int c = 0; c < G / 16; ++c) {
+                        const int k = 32 * c + lane;  // 32-byte piece k of the warp's rows
+                        const uint32_t* src = wrows + (k / (G / 16)) * kRowWords + 8 * (k % (G / 16));
+                        const uint4 a = *reinterpret_cast<const uint4*>(src);
+                        const uint4 b = *reinterpret_cast<const uint4*>(src + 4);
+                        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+                        store16<WIDE>(reinterpret_cast<uint16_t*>(d0) + 16 * k, wa, wb);
+                    }
+                    __syncwarp();  // the rows are read before the lanes stage their next ones
+                } else {
+#pragma unroll
+                    for (int c = 0; c < G / 16; ++c) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(row + 8 * c);
+                        const uint4 b = *reinterpret_cast<const uint4*>(row + 8 * c + 4);
+                        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+                        store16<WIDE>(dst + 16 * c, wa, wb);
+                    }
                 }
             }
         }
