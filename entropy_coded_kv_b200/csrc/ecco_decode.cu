@@ -46,14 +46,6 @@ constexpr size_t dec_smem()
            (G == kG ? 0 : (size_t)dec_threads<G>() * kRowWords * 4);
 }
 
-// 32 bytes from global memory through the read-only path (one 256-bit load).
-__device__ __forceinline__ void ldg_nc_v8(const void* p, uint4& a, uint4& b)
-{
-    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                 : "l"(p));
-}
-
 // WIDE: blocks and output both 32-byte aligned: 32-byte block loads and
 // stores (a 64-byte block in two loads: 2.7% faster on the long-context
 // cache than four 16-byte loads); else 16-byte loads and stores.

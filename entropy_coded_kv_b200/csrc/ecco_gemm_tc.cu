@@ -169,6 +169,7 @@ struct TcArgs {
     int* flag;  // host-visible timeout flag (mapped pinned memory), or null
     int64_t rows, gpr, cols, units;
     int batch;
+    bool wide;  // blocks 32-byte aligned
 };
 
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_constant__ TcArgs A)
@@ -294,18 +295,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         // ---- this thread's row block (and the next unit's on its way to L2)
         const int64_t row = rt * kTcThreads + tid;
         const bool row_ok = row < A.rows;
-        if (l + 1 < nu) {
-            const int64_t un = u + 1, rn = (un / A.gpr) * kTcThreads + tid;
+        if (l + 1 < nu) {  // the next unit: the next column group, or the next row tile's first
+            const bool wrap = g + 1 == A.gpr;
+            const int64_t rn = row + (wrap ? kTcThreads : 0), gn = wrap ? 0 : g + 1;
             if (rn < A.rows)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(A.blocks + (rn * A.gpr + (un % A.gpr)) * ECCO_BLOCK_BYTES));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(A.blocks + (rn * A.gpr + gn) * ECCO_BLOCK_BYTES));
         }
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0, q2 = q0, q3 = q0;
         if (row_ok) {
             const uint8_t* src = A.blocks + (row * A.gpr + g) * ECCO_BLOCK_BYTES;
-            q0 = ldg_nc_v4(src);
-            q1 = ldg_nc_v4(src + 16);
-            q2 = ldg_nc_v4(src + 32);
-            q3 = ldg_nc_v4(src + 48);
+            if (A.wide) {  // 32-byte aligned blocks: two 32-byte loads
+                ldg_nc_v8(src, q0, q1);
+                ldg_nc_v8(src + 32, q2, q3);
+            } else {
+                q0 = ldg_nc_v4(src);
+                q1 = ldg_nc_v4(src + 16);
+                q2 = ldg_nc_v4(src + 32);
+                q3 = ldg_nc_v4(src + 48);
+            }
         }
         const uint32_t code = q0.x & 0xffu;
         const int p = (int)((q0.x >> 8) & 63u);
@@ -447,6 +454,7 @@ cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t 
     A.cols = cols;
     A.units = (rows + kTcThreads - 1) / kTcThreads * A.gpr;
     A.batch = batch;
+    A.wide = (reinterpret_cast<uintptr_t>(blocks) & 31u) == 0;
     const int64_t sms = device_sm_count();
     const int grid = (int)(A.units < sms ? A.units : sms);  // one resident CTA per SM, balanced unit ranges
     gemm_tc_kernel<<<grid, kTcThreads, kTcSmem, s>>>(A);

@@ -168,6 +168,15 @@ __device__ __forceinline__ bool scale_code_is_null(uint32_t code)
     return mag == 0u || mag == 0x7fu;
 }
 
+// 32 bytes from global memory through the read-only path (one 256-bit load;
+// p 32-byte aligned).
+__device__ __forceinline__ void ldg_nc_v8(const void* p, uint4& a, uint4& b)
+{
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p)
 {
     uint4 r;
