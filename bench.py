@@ -1256,11 +1256,18 @@ KERNEL_SOURCES = {
 
 
 def source_hash(files) -> str:
+    """Hash of the files' code: comments and blank lines are left out, so a
+    comment edit keeps a capture valid while any code change voids it."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "entropy_coded_kv_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "entropy_coded_kv_b200", "csrc", f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

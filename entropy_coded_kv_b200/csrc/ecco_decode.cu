@@ -7,8 +7,9 @@
 // B200 has millions of independent blocks in flight instead, so here every
 // thread walks one block's stream serially and parallelism comes from the
 // blocks: the serial chain (one shared-memory table lookup per symbol) is
-// hidden by 32 resident warps per SM, and no work is spent on offsets that
-// turn out to be wrong.
+// hidden by 28 resident warps per SM, and no work is spent on offsets that
+// turn out to be wrong.  (ecco_decode_spec.cu builds the page's speculative
+// scheme on a warp per block, for comparison: it is several times slower.)
 //
 // G = 64 is the activation format (64 values per 512-bit block, the review
 // page's 2x ratio for activations); everything else is shared.  Activation
@@ -20,7 +21,8 @@
 // Per block: parse the header (scale code, pattern, codebook), form the 16
 // output values bf16(s * C[p][j]) as register byte planes, decode the stream
 // 8 symbols at a time (ecco_block.cuh), write each 16 decoded values with one
-// 32-byte store, then apply the outlier records of an unclipped stream.
+// 32-byte store (lane pairs write 64 contiguous bytes of one row per
+// instruction), then apply the outlier records of an unclipped stream.
 #include <algorithm>
 
 #include "ecco_block.cuh"

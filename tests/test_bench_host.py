@@ -39,6 +39,19 @@ def test_traffic_is_reported_only_while_the_sources_are_unchanged(monkeypatch):
     assert bench.traffic_for("kv", "no_such_kernel") is None
 
 
+def test_source_hash_follows_code_not_comments(tmp_path, monkeypatch):
+    d = tmp_path / "entropy_coded_kv_b200" / "csrc"
+    d.mkdir(parents=True)
+    f = d / "k.cu"
+    f.write_text("// header\nint a = 1; /* note */\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.source_hash(["k.cu"])
+    f.write_text("// a longer header\n/* two\n   lines */\n\nint a = 1;   // why\n")
+    assert bench.source_hash(["k.cu"]) == h0
+    f.write_text("int a = 2;\n")
+    assert bench.source_hash(["k.cu"]) != h0
+
+
 def test_source_hash_covers_every_listed_file():
     for kernel, files in bench.KERNEL_SOURCES.items():
         for f in files:
