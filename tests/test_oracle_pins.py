@@ -349,6 +349,20 @@ def check_group(blob, x, gs: int = 128):
     e64 = (np.float64(umin) - C[:, 0]) ** 2 + (np.float64(umax) - C[:, 14]) ** 2
     assert e64[gi.p] <= e64.min() * (1 + 1e-5) + 1e-30
     assert not np.any(e64[: gi.p] < e64[gi.p] * (1 - 1e-5))
+    # ... and exactly R8: every operation rounded to fp32 (numpy float32
+    # arithmetic, no fused multiply-add), the first pattern with the least error
+    C32 = np.asarray(C, dtype=np.float32)
+    d0 = np.float32(umin) - C32[:, 0]
+    d1 = np.float32(umax) - C32[:, 14]
+    e32 = (d0 * d0) + (d1 * d1)
+    assert e32.dtype == np.float32
+    assert gi.p == int(np.flatnonzero(e32 == e32.min())[0])
+    # quantisation exactly by R9: the count of fp32 thresholds
+    # T_j = fp32(fp32(C_j + C_j+1) * 0.5) strictly below u
+    T32 = (C32[gi.p, :-1] + C32[gi.p, 1:]) * np.float32(0.5)
+    assert T32.dtype == np.float32
+    for i in others:
+        assert gi.sym[i] == int(np.count_nonzero(T32 < np.float32(u[i]))), i
     # quantisation: nearest centroid of the chosen pattern (midpoints excepted)
     cp = C[gi.p].astype(np.float64)
     for i in others:
