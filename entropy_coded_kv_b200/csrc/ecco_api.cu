@@ -232,7 +232,9 @@ namespace {
 constexpr size_t kScratchAlign = 256;
 size_t staged_partials_bytes(int batch, int kv_heads, int group, int seq_len)
 {
-    const size_t p = ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len);
+    if (ecco_decode_attention_workspace_bytes(batch, kv_heads, group, seq_len) == 0) return 0;
+    const size_t p = sizeof(float) * 130 * (size_t)batch * (size_t)kv_heads * (size_t)group *
+                     (size_t)ecco::attention_staged_splits(seq_len);
     return (p + kScratchAlign - 1) / kScratchAlign * kScratchAlign;
 }
 }  // namespace

@@ -27,6 +27,8 @@
 // added as (new - old) * q on the score and p * (new - old) on the output.
 // Partial (max, sum, p.V) of every split go to a caller-owned workspace; a
 // second kernel merges the splits with the usual log-sum-exp rescaling.
+// The staged variant reads rows the block decoder has already written and
+// takes 256-token splits (8 warps per CTA) instead.
 #include <atomic>
 
 #include "ecco_block.cuh"
@@ -37,6 +39,10 @@ namespace {
 constexpr int kAtThreads = 512;
 constexpr int kAtWarps = kAtThreads / 32;
 constexpr int kAtStride = kAtThreads;
+// The staged split kernel: 8 warps, 256 tokens per split, so that three CTAs
+// (row tiles and q: 71 KB of shared memory each) are resident per SM.
+constexpr int kStWarps = 8;
+constexpr int kStTokens = kStWarps * 32;
 constexpr int kStageRow = 20;  // words per staged token row: 32 bf16 + 16 B pad (ldmatrix conflict-free)
 constexpr int kHeads = 8;      // rows 0-7 of an m16 tile: the query heads of one KV head
 constexpr int kQbRow = 136;    // bf16 per staged q row (padded: conflict-free fragment loads)
@@ -52,8 +58,8 @@ struct AttnArgs {
     float scale;
     float* ws;  // [B][H*G][splits][130]: 128 partial p.V, then max, sum
     // Staged path only: the current chunk's decoded K and V rows (bf16,
-    // [B*H][cstride][128]), its first token c0 (a multiple of 512) and the
-    // index of its first split.
+    // [B*H][cstride][128]), its first token c0 (a multiple of kStTokens) and
+    // the index of its first split.
     const uint16_t* kx;
     const uint16_t* vx;
     int64_t c0, cstride;
@@ -73,24 +79,25 @@ constexpr size_t kOffRed = kOffQb + (size_t)kHeads * kQbRow * 2;              //
 constexpr size_t kOffAcc = kOffRed + (size_t)2 * kAtWarps * kHeads * 4;       // [head][128] f32
 constexpr size_t kAttnSmem = kOffAcc + (size_t)kHeads * 128 * 4 + kSmemAlign;
 static_assert(kOffQb % 16 == 0 && kOffRed % 16 == 0 && kOffAcc % 16 == 0, "alignment");
-// Staged path: no tables, stream words or nibbles; each warp's tile holds its
-// 32 tokens' whole decoded rows (filled by cp.async), 272 B apart so that
-// ldmatrix rows fall on distinct banks, and each warp writes its P . V to its
-// own slice, summed over the warps once (no shared-memory atomics: 16 warps
-// adding into one accumulator was measured 9-16% slower per call).
+// Staged path: no tables, stream words, nibbles or f32 copies of q; each
+// warp's tile holds its 32 tokens' whole decoded rows (filled by cp.async),
+// 272 B apart so that ldmatrix rows fall on distinct banks.  Once a warp has
+// read a quarter of its V rows (dims 32 qd ..), it writes its P . V for those
+// dims into the same columns of its own tile (head g in rows 2g and 2g + 1),
+// and the warps' slices are summed once into the partial result (no
+// shared-memory atomics: 16 warps adding into one accumulator was measured
+// 9-16% slower per call).  71 KB per CTA: three CTAs of 8 warps per SM.
 constexpr int kFullRow = 68;  // words per staged full row: 128 bf16 + 16 B pad
 constexpr size_t kSOffTile = 0;
-constexpr size_t kSOffQf = kSOffTile + (size_t)kAtWarps * 32 * kFullRow * 4;
-constexpr size_t kSOffQb = kSOffQf + (size_t)kHeads * 128 * 4;
+constexpr size_t kSOffQb = kSOffTile + (size_t)kStWarps * 32 * kFullRow * 4;
 constexpr size_t kSOffRed = kSOffQb + (size_t)kHeads * kQbRow * 2;
-constexpr size_t kSOffAcc = kSOffRed + (size_t)2 * kAtWarps * kHeads * 4;
-constexpr size_t kSOffPart = kSOffAcc + (size_t)kHeads * 128 * 4;  // [warp][head][128] f32
-constexpr size_t kAttnSmemStaged = kSOffPart + (size_t)kAtWarps * kHeads * 128 * 4 + kSmemAlign;
-static_assert(kSOffQb % 16 == 0 && kSOffRed % 16 == 0 && kSOffAcc % 16 == 0 && kSOffPart % 16 == 0, "alignment");
+constexpr size_t kAttnSmemStaged = kSOffRed + (size_t)2 * kStWarps * kHeads * 4 + kSmemAlign;
+static_assert(kSOffQb % 16 == 0 && kSOffRed % 16 == 0, "alignment");
+static_assert(3 * (kAttnSmemStaged + 1024) <= 233472, "three staged CTAs per SM");
 
 // Tokens per chunk of the staged path: the decoded K and V rows of a chunk
 // (2 x rows x chunk x 256 B) stay within kStagedScratchBytes; a multiple of
-// 512 (whole splits).  Measured on B200 ([8, 8, 4096] and [1, 8, 131072]
+// 512 (whole splits of either kernel).  Measured on B200 ([8, 8, 4096] and [1, 8, 131072]
 // caches): chunks that fit in L2 (32 MiB) are slower than one large chunk,
 // because a decoder launch needs several blocks per thread to hide its serial
 // walk, so the bound is set by memory use, not by L2.
@@ -227,22 +234,32 @@ __device__ __forceinline__ void k_quarter_mma(float (&S)[4][4], const uint32_t* 
     }
 }
 
-// part[head][dims 32 qd ..] = P . V over the warp's 32 staged tokens (this
-// warp's own slice: plain stores).
+// P . V over the warp's 32 staged tokens for dims 32 qd .. 32 qd + 31, written
+// over those dims' columns of the warp's own tile once every lane has read
+// them: head g's 32 sums go to rows 2g (dims 0-15) and 2g + 1 (dims 16-31),
+// words 16 qd .. 16 qd + 15 (plain stores; no other warp touches the tile).
 template <int G>
-__device__ __forceinline__ void v_quarter_part(float* part, const uint32_t (&pa)[2][4], uint32_t stage_sh, int lane,
+__device__ __forceinline__ void v_quarter_part(float* tile, const uint32_t (&pa)[2][4], uint32_t stage_sh, int lane,
                                                int gid, int tig, int qd)
 {
+    uint32_t bfr[4][4];
+#pragma unroll
+    for (int nd = 0; nd < 4; ++nd) ldsm_x4_t(stage_sh + (uint32_t)((lane * kFullRow + nd * 4) * 4), bfr[nd]);
+    float o[4][4];
 #pragma unroll
     for (int nd = 0; nd < 4; ++nd) {
-        uint32_t bfr[4];
-        ldsm_x4_t(stage_sh + (uint32_t)((lane * kFullRow + nd * 4) * 4), bfr);
-        float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        mma_bf16(o, pa[0][0], pa[0][1], pa[0][2], pa[0][3], bfr[0], bfr[1]);
-        mma_bf16(o, pa[1][0], pa[1][1], pa[1][2], pa[1][3], bfr[2], bfr[3]);
-        if (gid < G) {
-            const int d = qd * 32 + nd * 8 + 2 * tig;
-            *reinterpret_cast<float2*>(part + gid * 128 + d) = make_float2(o[0] + o[2], o[1] + o[3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nd][e] = 0.0f;
+        mma_bf16(o[nd], pa[0][0], pa[0][1], pa[0][2], pa[0][3], bfr[nd][0], bfr[nd][1]);
+        mma_bf16(o[nd], pa[1][0], pa[1][1], pa[1][2], pa[1][3], bfr[nd][2], bfr[nd][3]);
+    }
+    __syncwarp();  // the quarter's columns are read by every lane
+    if (gid < G) {
+#pragma unroll
+        for (int nd = 0; nd < 4; ++nd) {
+            const int dd = nd * 8 + 2 * tig;  // dim within the quarter
+            *reinterpret_cast<float2*>(tile + (2 * gid + (dd >> 4)) * kFullRow + 16 * qd + (dd & 15)) =
+                make_float2(o[nd][0] + o[nd][2], o[nd][1] + o[nd][3]);
         }
     }
 }
@@ -277,8 +294,11 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)
 // STAGED = true: the split's rows were decoded into A.kx / A.vx by the block
 // decoder just before (records already applied), and are read from there.
 template <int G, bool STAGED>
-__global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_constant__ AttnArgs A)
+__global__ void __launch_bounds__(STAGED ? kStTokens : kAtThreads, STAGED ? 3 : 1)
+    attn_split_kernel(const __grid_constant__ AttnArgs A)
 {
+    constexpr int W = STAGED ? kStWarps : kAtWarps;  // warps, 32 tokens each
+    constexpr int NT = W * 32;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t* smem = aligned_smem(smem_raw);
     // unstaged only: tables, stream words, nibbles, per-token exchange
@@ -286,27 +306,29 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
     float* s_Ct = reinterpret_cast<float*>(smem + kOffCt);
     uint32_t* s_w = reinterpret_cast<uint32_t*>(smem + kOffWords);
     float* s_x = reinterpret_cast<float*>(smem + kOffX);
-    float* s_qf = reinterpret_cast<float*>(smem + (STAGED ? kSOffQf : kOffQf));
+    float* s_qf = reinterpret_cast<float*>(smem + kOffQf);    // unstaged only
+    float* s_acc = reinterpret_cast<float*>(smem + kOffAcc);  // unstaged only
     uint16_t* s_qb = reinterpret_cast<uint16_t*>(smem + (STAGED ? kSOffQb : kOffQb));
     float* s_red = reinterpret_cast<float*>(smem + (STAGED ? kSOffRed : kOffRed));
-    float* s_acc = reinterpret_cast<float*>(smem + (STAGED ? kSOffAcc : kOffAcc));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;  // mma fragment coordinates
     const int split = (STAGED ? A.split0 : 0) + (int)blockIdx.x, bh = blockIdx.y;
     const int b = bh / A.H, h = bh - b * A.H;
     const int Hq = A.H * G;
-    const int tok0 = split * kAtThreads + warp * 32;  // first token of this warp
+    const int tok0 = split * NT + warp * 32;  // first token of this warp
     const bool have = tok0 + lane < A.S;
     const int64_t blk = (int64_t)bh * A.s_cap + tok0 + lane;
 
     // q of the group's heads (rows >= G are zero), accumulator cleared
-    for (int i = tid; i < kHeads * 128; i += kAtThreads) {
+    for (int i = tid; i < kHeads * 128; i += NT) {
         const int g = i >> 7, d = i & 127;
         const uint16_t v = (g < G) ? A.q[((int64_t)b * Hq + h * G + g) * 128 + d] : (uint16_t)0;
         s_qb[g * kQbRow + d] = v;
-        s_qf[i] = bf16_bits_to_f32(v);
-        s_acc[i] = 0.0f;
+        if constexpr (!STAGED) {
+            s_qf[i] = bf16_bits_to_f32(v);
+            s_acc[i] = 0.0f;
+        }
     }
     if constexpr (!STAGED) stage_tables<kAtThreads>(A.ktb, s_lut, s_Ct, tid);
     __syncthreads();
@@ -392,7 +414,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
     __syncthreads();
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kAtWarps; ++w) M = fmaxf(M, s_red[w * kHeads + gid]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, s_red[w * kHeads + gid]);
     float sum = 0.0f;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
@@ -405,11 +427,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
         }
     sum += __shfl_xor_sync(0xffffffffu, sum, 1);
     sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    if (tig == 0) s_red[kAtWarps * kHeads + warp * kHeads + gid] = sum;
+    if (tig == 0) s_red[W * kHeads + warp * kHeads + gid] = sum;
     __syncthreads();  // also: the K tables are no longer read
     float L = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kAtWarps; ++w) L += s_red[kAtWarps * kHeads + w * kHeads + gid];
+    for (int w = 0; w < W; ++w) L += s_red[W * kHeads + w * kHeads + gid];
     if constexpr (!STAGED) stage_tables<kAtThreads>(A.vtb, s_lut, s_Ct, tid);
 
     // A fragments of P, k-step ks = tokens 16 ks + (0..15):
@@ -426,22 +448,25 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
             pa[ks][2 * half + 1] = pack2_bf16(r0, r1);
         }
     }
-    __syncthreads();
+    if constexpr (!STAGED) __syncthreads();  // the V tables are staged
 
-    // ---------------- V pass: O = P V
+    // ---------------- V pass: O = P V, and this split's partial result
+    float* out = A.ws + ((int64_t)b * Hq + h * G) * A.splits * 130;
     if constexpr (STAGED) {
         stage_rows_wait();
         __syncwarp();  // other lanes' copies landed too
-        float* part = reinterpret_cast<float*>(smem + kSOffPart) + warp * kHeads * 128;
+        float* tiles = reinterpret_cast<float*>(smem + kSOffTile);
 #pragma unroll
-        for (int qd = 0; qd < 4; ++qd) v_quarter_part<G>(part, pa, tile_sh + 64u * qd, lane, gid, tig, qd);
+        for (int qd = 0; qd < 4; ++qd)
+            v_quarter_part<G>(tiles + warp * 32 * kFullRow, pa, tile_sh + 64u * qd, lane, gid, tig, qd);
         __syncthreads();
-        for (int i = tid; i < G * 128; i += kAtThreads) {
-            const float* pp = reinterpret_cast<const float*>(smem + kSOffPart) + i;
+        for (int i = tid; i < G * 128; i += NT) {
+            const int g = i >> 7, d = i & 127, dd = d & 31;
+            const float* pp = tiles + (2 * g + (dd >> 4)) * kFullRow + 16 * (d >> 5) + (dd & 15);
             float acc = 0.0f;
 #pragma unroll
-            for (int w = 0; w < kAtWarps; ++w) acc += pp[w * kHeads * 128];
-            s_acc[i] = acc;
+            for (int w = 0; w < W; ++w) acc += pp[w * 32 * kFullRow];
+            out[((int64_t)g * A.splits + split) * 130 + d] = acc;
         }
     } else {
         uint4 q0, q1, q2, q3;
@@ -462,14 +487,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_split_kernel(const __grid_
 #pragma unroll
             for (int g = 0; g < G; ++g) atomicAdd(&s_acc[g * 128 + i], pt[g] * dv);
         });
-    }
-    __syncthreads();
-
-    // ---------------- this split's partial result
-    float* out = A.ws + ((int64_t)b * Hq + h * G) * A.splits * 130;
-    for (int i = tid; i < G * 128; i += kAtThreads) {
-        const int g = i >> 7, d = i & 127;
-        out[((int64_t)g * A.splits + split) * 130 + d] = s_acc[i];
+        __syncthreads();
+        for (int i = tid; i < G * 128; i += NT) {
+            const int g = i >> 7, d = i & 127;
+            out[((int64_t)g * A.splits + split) * 130 + d] = s_acc[i];
+        }
     }
     if (warp == 0 && tig == 0 && gid < G) {
         out[((int64_t)gid * A.splits + split) * 130 + 128] = M;
@@ -536,9 +558,9 @@ cudaError_t run_attn_staged(AttnArgs A, int B, const ecco_tables* kt, const ecco
         e = launch_decode_multi(seg, 2, s);
         if (e != cudaSuccess) return e;
         A.c0 = c0;
-        A.split0 = (int)(c0 / kAtThreads);
-        dim3 grid((unsigned)((cn + kAtThreads - 1) / kAtThreads), (unsigned)rows);
-        attn_split_kernel<G, true><<<grid, kAtThreads, kAttnSmemStaged, s>>>(A);
+        A.split0 = (int)(c0 / kStTokens);
+        dim3 grid((unsigned)((cn + kStTokens - 1) / kStTokens), (unsigned)rows);
+        attn_split_kernel<G, true><<<grid, kStTokens, kAttnSmemStaged, s>>>(A);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -549,6 +571,8 @@ cudaError_t run_attn_staged(AttnArgs A, int B, const ecco_tables* kt, const ecco
 }  // namespace
 
 int attention_splits(int seq_len) { return (seq_len + kAtThreads - 1) / kAtThreads; }
+
+int attention_staged_splits(int seq_len) { return (seq_len + kStTokens - 1) / kStTokens; }
 
 int64_t staged_chunk_tokens(int B, int H, int seq_len)
 {
@@ -582,7 +606,8 @@ cudaError_t launch_attention_staged(const ecco_tables* kt, const ecco_tables* vt
                                     const uint16_t* q, float scale, float* out, float* ws, uint16_t* scratch,
                                     cudaStream_t s)
 {
-    AttnArgs A{kt->d, vt->d, kblk, vblk, s_cap, H, G, S, attention_splits(S), q, scale, ws, nullptr, nullptr, 0, 0, 0};
+    AttnArgs A{kt->d, vt->d, kblk, vblk, s_cap, H, G, S, attention_staged_splits(S), q, scale, ws,
+               nullptr, nullptr, 0, 0, 0};
     switch (G) {
         case 1: return run_attn_staged<1>(A, B, kt, vt, scratch, s, out);
         case 2: return run_attn_staged<2>(A, B, kt, vt, scratch, s, out);

@@ -96,7 +96,8 @@ cudaError_t launch_decode_act(const ecco_tables* t, const uint8_t* blocks, const
 cudaError_t launch_encode_multi(const ecco_segment* segs, int n, ecco_stats* stats,
                                 cudaStream_t s);
 
-// Attention over a compressed KV cache: splits of 512 tokens, then a merge.
+// Attention over a compressed KV cache: splits of 512 tokens (the fused
+// kernel), then a merge.
 int attention_splits(int seq_len);
 cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
                              const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
@@ -109,6 +110,9 @@ cudaError_t launch_attention(const ecco_tables* kt, const ecco_tables* vt, const
 // stream words and tiles leave it half the decoder's resident warps, so its
 // serial walk shows through.
 int64_t staged_chunk_tokens(int B, int H, int seq_len);
+// Splits of the staged path's kernel (256 tokens each): its partials hold
+// 130 floats per (batch, query head, split).
+int attention_staged_splits(int seq_len);
 cudaError_t launch_attention_staged(const ecco_tables* kt, const ecco_tables* vt, const uint8_t* kblk,
                                     const uint8_t* vblk, int64_t s_cap, int B, int H, int G, int S,
                                     const uint16_t* q, float scale, float* out, float* ws, uint16_t* scratch,

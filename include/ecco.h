@@ -238,8 +238,9 @@ int ecco_decode_attention(const ecco_tables* k_tables, const ecco_tables* v_tabl
  * stages: for each chunk of tokens the block decoder (ecco_decode_multi's
  * kernel) writes the chunk's decoded K and V rows to a scratch inside the
  * workspace, then a split kernel reads them back with coalesced copies.  A
- * chunk holds whole 512-token splits, and its rows (2 x batch x kv_heads x
- * chunk x 256 B) stay within 1 GiB, so most caches run as one chunk.  The
+ * chunk is a multiple of 512 tokens (whole 256-token splits), and its rows
+ * (2 x batch x kv_heads x chunk x 256 B) stay within 1 GiB, so most caches
+ * run as one chunk.  The
  * decoded rows cross HBM once each way; in exchange the decode runs at the
  * standalone decoder's occupancy, which the single fused kernel cannot reach
  * (its tables, stream words and tiles leave it half the resident warps).  The

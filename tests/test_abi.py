@@ -69,15 +69,16 @@ def test_argument_errors_need_no_gpu(lib):
     assert lib.ecco_decode_attention_workspace_bytes(1, 1, 1, 513) == 4 * 130 * 2
     assert lib.ecco_decode_attention_workspace_bytes(1, 1, 9, 10) == 0
     assert lib.ecco_decode_attention_workspace_bytes(1, 1, 1, 0) == 0
-    # staged: partials rounded up to 256 B, 256 B of slack, then K and V rows of
-    # one chunk (whole 512-token splits within 1 GiB, at most the sequence)
+    # staged: partials of 256-token splits rounded up to 256 B, 256 B of slack,
+    # then K and V rows of one chunk (a multiple of 512 tokens within 1 GiB, at
+    # most the sequence rounded up to 512)
     assert lib.ecco_decode_attention_staged_workspace_bytes(8, 8, 4, 4096) == (
-        4 * 130 * 8 * 8 * 4 * 8 + 256 + 2 * 64 * 4096 * 256)
+        4 * 130 * 8 * 8 * 4 * 16 + 256 + 2 * 64 * 4096 * 256)
     assert lib.ecco_decode_attention_staged_workspace_bytes(1, 8, 4, 131072) == (
-        4 * 130 * 8 * 4 * 256 + 256 + 2 * 8 * 131072 * 256)
+        4 * 130 * 8 * 4 * 512 + 256 + 2 * 8 * 131072 * 256)
     assert lib.ecco_decode_attention_staged_workspace_bytes(64, 32, 1, 8192) == (
-        4 * 130 * 64 * 32 * 16 + 256 + 2 * 64 * 32 * 1024 * 256)
-    assert lib.ecco_decode_attention_staged_workspace_bytes(1, 1, 1, 513) == 1280 + 256 + 2 * 1024 * 256
+        4 * 130 * 64 * 32 * 32 + 256 + 2 * 64 * 32 * 1024 * 256)
+    assert lib.ecco_decode_attention_staged_workspace_bytes(1, 1, 1, 513) == 1792 + 256 + 2 * 1024 * 256
     assert lib.ecco_decode_attention_staged_workspace_bytes(1, 1, 9, 10) == 0
     assert lib.ecco_decode_attention_staged(None, None, None, None, 64, 1, 1, 1, 1, None, 1.0, None, None, 0,
                                             None) == _lib.ECCO_ERR_ARG

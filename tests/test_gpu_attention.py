@@ -89,10 +89,10 @@ def test_attention_matches_oracle(B, H, G, S_cap, n, ktn, vtn, kk, vk, path):
 def test_staged_chunks():
     """4096 (batch, KV head) rows make the staged chunk 512 tokens (1 GiB of
     decoded rows), so 1237 tokens run as chunks of 512, 512 and 213 tokens
-    through the same scratch."""
+    through the same scratch; the partials hold five 256-token splits."""
     B, H, G, S_cap, n = 512, 8, 1, 1240, 1237
     assert _lib.load().ecco_decode_attention_staged_workspace_bytes(B, H, G, n) == (
-        4 * 130 * B * H * G * 3 + 256 + 2 * B * H * 512 * 256)
+        4 * 130 * B * H * G * 5 + 256 + 2 * B * H * 512 * 256)
     kt, vt = table_set("learned_kv"), table_set("random2")
     rng = np.random.default_rng(31)  # every 64-byte pattern is a block (clips, records, null scales)
     kb = rng.integers(0, 256, (B, H, S_cap, 64), dtype=np.uint8)
