@@ -605,8 +605,10 @@ class LongCtxWorkload(Workload):
         self.out = [torch.empty_like(c) for c in self.caches]
         self.new = [c.view(8, self.S, 128)[:, self.S - 1:].contiguous() for c in self.caches]
         app = ecco.kv_append_desc(8, 1, self.S, self.S - 1)
-        self.app = [ecco.Seg(tb, nw, b, app) for tb, nw, b in zip(self.tables, self.new, self.blocks)]
-        self.dec = [ecco.Seg(tb, b, o.view(-1, 128)) for tb, b, o in zip(self.tables, self.blocks, self.out)]
+        # checked and marshalled once: a step only passes the prepared segments
+        self.app = ecco.prepare_encode([ecco.Seg(tb, nw, b, app) for tb, nw, b in zip(self.tables, self.new, self.blocks)])
+        self.dec_segs = [ecco.Seg(tb, b, o.view(-1, 128)) for tb, b, o in zip(self.tables, self.blocks, self.out)]
+        self.dec = ecco.prepare_decode(self.dec_segs)
         self.n = sum(c.numel() // 128 for c in self.caches)
         self.launches_per_step = 2
         self.ev = {"encode": [], "decode": []}
@@ -656,8 +658,8 @@ class LongCtxWorkload(Workload):
         for i in range(0, len(self.caches), 2):
             ins = [(self.h_blocks[j], self.blocks[j]) for j in (i, i + 1)] + \
                   [(self.h_new[j], self.d_new[j]) for j in (i, i + 1)]
-            layers.append((ins, (lambda a, b: lambda: (e.encode_multi(a), e.decode_multi(b)))(e2e_app[i:i + 2],
-                                                                                           self.dec[i:i + 2]),
+            layers.append((ins, (lambda a, b: lambda: (e.encode_multi(a), e.decode_multi(b)))(
+                               e.prepare_encode(e2e_app[i:i + 2]), e.prepare_decode(self.dec_segs[i:i + 2])),
                            self.out[i:i + 2]))
         self.stream = LayerStream(torch, self.dev, layers)
         self.h2d, self.d2h = self.stream.h2d, self.stream.d2h

@@ -24,6 +24,7 @@ GROUP_ACT = 64  # activation format: 64 values per 64-byte block
 BLOCK_BYTES = 64
 
 __all__ = ["Tables", "encode", "decode", "decode_gemv", "decode_multi", "encode_multi",
+           "Prepared", "prepare_encode", "prepare_decode",
            "decode_attention", "attention_workspace_bytes", "decode_attention_static",
            "decode_attention_staged", "attention_staged_workspace_bytes",
            "encode_act", "decode_act", "GROUP_ACT", "learn_tables", "huffman_lengths",
@@ -336,20 +337,57 @@ def _segments(segs, src_dtype, dst_dtype, src_unit, dst_unit):
     return arr
 
 
-def decode_multi(segs: list[Seg]) -> None:
-    if not segs:
+class Prepared:
+    """Segments checked and marshalled once, for a multi-segment call repeated
+    on the same buffers (a per-token KV append over every layer): the call then
+    only passes the prepared array and the current stream.  It keeps the
+    tensors and tables alive; their contents may change between calls, their
+    storage may not."""
+
+    def __init__(self, segs: list[Seg], kind: str):
+        if kind not in ("encode", "decode"):
+            raise ValueError("kind is 'encode' or 'decode'")
+        self.kind, self.segs = kind, list(segs)
+        if kind == "encode":
+            self.arr = _segments(self.segs, torch.bfloat16, torch.uint8, GROUP, BLOCK_BYTES)
+        else:
+            self.arr = _segments(self.segs, torch.uint8, torch.bfloat16, BLOCK_BYTES, GROUP)
+        self.device = self.segs[0].tables.device if self.segs else None
+
+    def __len__(self):
+        return len(self.segs)
+
+
+def prepare_encode(segs: list[Seg]) -> Prepared:
+    return Prepared(segs, "encode")
+
+
+def prepare_decode(segs: list[Seg]) -> Prepared:
+    return Prepared(segs, "decode")
+
+
+def _marshalled(segs, kind, src_dtype, dst_dtype, src_unit, dst_unit):
+    if isinstance(segs, Prepared):
+        if segs.kind != kind:
+            raise ValueError(f"segments prepared for {segs.kind}, not {kind}")
+        return segs.arr, len(segs), segs.device
+    return _segments(segs, src_dtype, dst_dtype, src_unit, dst_unit), len(segs), segs[0].tables.device
+
+
+def decode_multi(segs: list[Seg] | Prepared) -> None:
+    if not len(segs):
         return
-    arr = _segments(segs, torch.uint8, torch.bfloat16, BLOCK_BYTES, GROUP)
-    rc = _lib.load().ecco_decode_multi(arr, len(segs), _stream(segs[0].tables.device))
+    arr, n, dev = _marshalled(segs, "decode", torch.uint8, torch.bfloat16, BLOCK_BYTES, GROUP)
+    rc = _lib.load().ecco_decode_multi(arr, n, _stream(dev))
     _lib.check(rc, "ecco_decode_multi")
 
 
-def encode_multi(segs: list[Seg], stats: torch.Tensor | None = None) -> None:
-    if not segs:
+def encode_multi(segs: list[Seg] | Prepared, stats: torch.Tensor | None = None) -> None:
+    if not len(segs):
         return
-    arr = _segments(segs, torch.bfloat16, torch.uint8, GROUP, BLOCK_BYTES)
+    arr, n, dev = _marshalled(segs, "encode", torch.bfloat16, torch.uint8, GROUP, BLOCK_BYTES)
     sp = ctypes.c_void_p(stats.data_ptr()) if stats is not None else None
-    rc = _lib.load().ecco_encode_multi(arr, len(segs), sp, _stream(segs[0].tables.device))
+    rc = _lib.load().ecco_encode_multi(arr, n, sp, _stream(dev))
     _lib.check(rc, "ecco_encode_multi")
 
 

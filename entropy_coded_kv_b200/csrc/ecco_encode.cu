@@ -502,6 +502,10 @@ cudaError_t run_encode(const EncParams<MAXSEG>& P, int select, cudaStream_t s)
 {
     const int per_cta = (32 / (G / 8)) * kEncWarps;
     int64_t want = (P.total + per_cta - 1) / per_cta;
+    // At least a CTA per segment: in a small launch of many small segments (a
+    // one-token KV append over every layer) a CTA would otherwise cross
+    // segments and stage each one's tables in turn, on its critical path.
+    if (want < P.n_seg) want = P.n_seg;
     int64_t cap = (int64_t)device_sm_count() * kEncCtasPerSm;  // one wave of resident CTAs
     int grid = (int)(want < cap ? want : cap);
     if constexpr (G == kG) {  // the full-MSE selection is offered for 128-value groups

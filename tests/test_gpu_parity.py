@@ -406,6 +406,40 @@ def test_multi_segment_many_small_segments_cross_launches():
     assert ecco.read_stats(st)["n_groups"] == tot
 
 
+def test_prepared_segments_one_token_append_over_64_segments():
+    """A one-token append into 64 caches of 16 rows (one CTA per segment),
+    through a prepared segment list called twice with new token contents:
+    bit-exact with the oracle, the other tokens untouched; a prepared decode
+    of the caches; a list prepared for decode is refused by encode_multi."""
+    names = ["learned_kv", "random1"]
+    tabs = [ecco.Tables(table_set(n), DEV) for n in names]
+    S, n = 5, 64
+    H = 16  # rows (KV heads) per cache: the "special" inputs need 9 groups or more
+    caches = [torch.zeros((H * S, 64), dtype=torch.uint8, device=DEV) for _ in range(n)]
+    new = [torch.empty((H, 128), dtype=torch.bfloat16, device=DEV) for _ in range(n)]
+    app = ecco.kv_append_desc(H, 1, S, S - 1)
+    prep = ecco.prepare_encode([ecco.Seg(tabs[i % 2], new[i], caches[i], app) for i in range(n)])
+    for rep in range(2):
+        xbs = [inputs(KINDS[(i + rep) % len(KINDS)], H, seed=100 * rep + i) for i in range(n)]
+        for nw, xb in zip(new, xbs):
+            nw.copy_(to_dev_bf16(xb).view(H, 128))
+        ecco.encode_multi(prep)
+        for i in range(n):
+            want, _ = oracle.encode(table_set(names[i % 2]), xbs[i], nthreads=2)
+            c = caches[i].view(H, S, 64).cpu().numpy()
+            np.testing.assert_array_equal(c[:, S - 1], want, err_msg=f"segment {i}, call {rep}")
+            assert not c[:, :S - 1].any()
+    ys = [torch.empty((H * S, 128), dtype=torch.bfloat16, device=DEV) for _ in range(n)]
+    dprep = ecco.prepare_decode([ecco.Seg(tabs[i % 2], caches[i], ys[i]) for i in range(n)])
+    ecco.decode_multi(dprep)
+    for i in (0, 1, n - 1):
+        blk = caches[i].cpu().numpy()
+        np.testing.assert_array_equal(bits(ys[i]).reshape(-1, 128), oracle.decode(table_set(names[i % 2]), blk,
+                                                                                 nthreads=2))
+    with pytest.raises(ValueError):
+        ecco.encode_multi(dprep)
+
+
 @pytest.mark.parametrize("batch", [5, 16])
 def test_tensor_core_gemv_one_hot_columns_are_exact(batch):
     """Batch > 4 runs on tcgen05 tensor cores.  With x[b] one-hot at column c_b,
