@@ -10,7 +10,10 @@
 // Work units are (row tile of 768 rows, one column group of 128 values); each
 // CTA (768 threads, one per SM) owns a balanced, contiguous range of units in
 // row-tile-major order, so consecutive units share a row tile and its
-// accumulators.  Thread t decodes row t's block of the unit with the block
+// accumulators.  When the units do not divide evenly over the CTAs and the
+// remainder is small, the remainder is not handed out whole (one more round
+// on a few SMs, the rest idle): its units are cut into warp steps of 32 rows,
+// which every CTA's first warps take after their whole units.  Thread t decodes row t's block of the unit with the block
 // walker of ecco_block.cuh.  The walk's speed comes from the warps running
 // freely (its latency is hidden by the other warps), so every warp feeds the
 // tensor cores on its own, with no barrier between warps inside a unit:
@@ -167,7 +170,8 @@ struct TcArgs {
     const uint16_t* x;
     float* y;
     int* flag;  // host-visible timeout flag (mapped pinned memory), or null
-    int64_t rows, gpr, cols, units;
+    int64_t rows, gpr, cols, units;  // units: whole units handed out to the CTAs
+    int64_t tail_steps;              // warp steps of the units left over (0: none)
     int batch;
     bool wide;  // blocks 32-byte aligned
 };
@@ -231,6 +235,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     bool acc = false;    // the warp's accumulators hold a partial sum
     const int64_t nu = u1 - u0;
     int64_t tile_row = (nu > 0) ? u0 / A.gpr : 0;
+    // Leftover units (when the units do not divide over the CTAs) are split
+    // into warp steps of 32 rows, kTcWarps per unit, and spread evenly: this
+    // CTA's steps [ts0, ts1) belong to at most two leftover units, its local
+    // units nu .. nl - 1 (their x goes through the ring like any unit's).
+    const int64_t ts0 = A.tail_steps * blockIdx.x / gridDim.x, ts1 = A.tail_steps * (blockIdx.x + 1) / gridDim.x;
+    const int64_t tl0 = ts0 / kTcWarps;
+    const int64_t nl = nu + ((ts1 > ts0) ? (ts1 - 1) / kTcWarps - tl0 + 1 : 0);
 
     // This thread's share of x for local unit l into its ring slot (l % 4),
     // after the unit that used the slot before (l - 4) has no MMA left; then
@@ -238,7 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     auto stage_x = [&](int64_t l) {
         const int slot = (int)(l % kBSlots);
         if (l >= kBSlots && ok) ok = mbar_wait(&bar_free[slot], (uint32_t)((l / kBSlots - 1) & 1), A.flag);
-        const int64_t g = (u0 + l) % A.gpr;
+        const int64_t g = (l < nu ? u0 + l : A.units + tl0 + (l - nu)) % A.gpr;
         uint8_t* Bw = s_B + slot * kBBytes;
         for (int e = tid; e < 16 * kG; e += kTcThreads) {
             const int b = e & 15, k = e >> 4;
@@ -255,7 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     };
     // Adds each thread's row of its warp's accumulators (plus the record
     // corrections) to y and starts the next row tile from zero.  Per warp.
-    auto flush = [&](int64_t rt) {
+    auto flush = [&](int64_t rt, int rb) {
         drain();
         ok = __all_sync(0xffffffffu, ok);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
             : "r"(taddr));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        const int64_t row = rt * kTcThreads + tid;
+        const int64_t row = rt * kTcThreads + rb + lane;
         if (ok && acc && row < A.rows) {
 #pragma unroll
             for (int b = 0; b < 16; ++b)
@@ -279,21 +290,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     };
 
-    for (int64_t l = 0; l < 2 && l < nu; ++l) stage_x(l);
-
-    for (int64_t l = 0; l < nu; ++l) {
-        const int64_t u = u0 + l;
-        const int64_t rt = u / A.gpr, g = u - rt * A.gpr;
-        if (rt != tile_row) {
-            flush(tile_row);
-            tile_row = rt;
-        }
-        if (l + 2 < nu) stage_x(l + 2);  // two units ahead
+    // One unit's work for this warp: its 32 rows rt * 768 + rb .. + 31 of
+    // column group g, x in ring slot l % 4.
+    auto run_unit = [&](int64_t l, int64_t rt, int64_t g, int rb) {
         const int slot = (int)(l % kBSlots);
         const uint8_t* B = s_B + slot * kBBytes;
 
         // ---- this thread's row block (and the next unit's on its way to L2)
-        const int64_t row = rt * kTcThreads + tid;
+        const int64_t row = rt * kTcThreads + rb + lane;
         const bool row_ok = row < A.rows;
         if (l + 1 < nu) {  // the next unit: the next column group, or the next row tile's first
             const bool wrap = g + 1 == A.gpr;
@@ -387,8 +391,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
         __syncwarp();  // the warp's lanes are done with this unit's x slot
         if (issuer)
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar_free[slot])) : "memory");
+    };
+
+    for (int64_t l = 0; l < 2 && l < nl; ++l) stage_x(l);
+
+    for (int64_t l = 0; l < nu; ++l) {
+        const int64_t u = u0 + l;
+        const int64_t rt = u / A.gpr, g = u - rt * A.gpr;
+        if (rt != tile_row) {
+            flush(tile_row, warp * 32);
+            tile_row = rt;
+        }
+        if (l + 2 < nl) stage_x(l + 2);  // two units ahead
+        run_unit(l, rt, g, warp * 32);
     }
-    flush(tile_row);
+    flush(tile_row, warp * 32);
+
+    // The CTA's leftover steps: warp w takes step ts0 + w (32 rows of a
+    // leftover unit), with the SM nearly to itself.
+    if (warp < ts1 - ts0) {
+        const int64_t j = ts0 + warp, tu = j / kTcWarps;
+        const int64_t u = A.units + tu, rt = u / A.gpr, g = u - rt * A.gpr;
+        const int rb = (int)(j - tu * kTcWarps) * 32;
+        run_unit(nu + (tu - tl0), rt, g, rb);
+        flush(rt, rb);
+    }
 
     // before the tensor memory is freed: the MMAs this warp committed are
     // done (bounded once more if a wait already gave up)
@@ -452,11 +479,18 @@ cudaError_t launch_gemm_tc(const ecco_tables* t, const uint8_t* blocks, int64_t 
     A.rows = rows;
     A.gpr = cols / kG;
     A.cols = cols;
-    A.units = (rows + kTcThreads - 1) / kTcThreads * A.gpr;
+    const int64_t units = (rows + kTcThreads - 1) / kTcThreads * A.gpr;
     A.batch = batch;
     A.wide = (reinterpret_cast<uintptr_t>(blocks) & 31u) == 0;
     const int64_t sms = device_sm_count();
-    const int grid = (int)(A.units < sms ? A.units : sms);  // one resident CTA per SM, balanced unit ranges
+    const int grid = (int)(units < sms ? units : sms);  // one resident CTA per SM, balanced unit ranges
+    // Units left over after whole rounds would take one more round on as many
+    // SMs while the rest idle; when they are at most a third of the grid they
+    // are split into warp steps spread over every CTA instead.
+    const int64_t left = units % grid;
+    const bool split = units > grid && left * 3 <= grid;
+    A.units = split ? units - left : units;
+    A.tail_steps = split ? left * kTcWarps : 0;
     gemm_tc_kernel<<<grid, kTcThreads, kTcSmem, s>>>(A);
     return cudaGetLastError();
 }

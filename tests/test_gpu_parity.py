@@ -459,6 +459,32 @@ def test_tensor_core_gemv_one_hot_columns_are_exact(batch):
         np.testing.assert_array_equal(y[b], (Wd[:, c].astype(np.uint32) << 16).view(np.float32))
 
 
+@pytest.mark.parametrize("batch", [5, 16])
+@pytest.mark.parametrize("rows,cols", [(1536, 9728), (58268, 256)])
+def test_tensor_core_gemv_leftover_units(batch, rows, cols):
+    """Shapes whose units (768 rows x one column group) do not divide evenly
+    over the SMs (152 units on 148, so a few CTAs take one unit more), the
+    extra units inside one row tile and across two row tiles with a ragged
+    last one.  One-hot columns come out bit for bit; random x stays within
+    the product tolerance."""
+    blob = table_set("learned_w")
+    wb = inputs("t5", rows * cols // 128, seed=rows)
+    blocks, _ = oracle.encode(blob, wb, nthreads=8)
+    Wd = oracle.decode(blob, blocks, nthreads=8).reshape(rows, cols)
+    t = ecco.Tables(blob, DEV)
+    dblocks = torch.from_numpy(blocks).to(DEV)
+    cs = [(37 * b + 5) % cols for b in range(batch - 1)] + [cols - 1]
+    x = np.zeros((batch, cols), dtype=np.uint16)
+    for b, c in enumerate(cs):
+        x[b, c] = 0x3F80
+    y = ecco.decode_gemv(dblocks, t, rows, cols, to_dev_bf16(x)).cpu().numpy()
+    for b, c in enumerate(cs):
+        np.testing.assert_array_equal(y[b], (Wd[:, c].astype(np.uint32) << 16).view(np.float32))
+    xb = bits(torch.randn(batch, cols, generator=torch.Generator().manual_seed(batch)).to(torch.bfloat16))
+    y = ecco.decode_gemv(dblocks, t, rows, cols, to_dev_bf16(xb)).cpu().numpy()
+    gemv_check(blob, blocks, rows, cols, xb, y)
+
+
 def test_no_device_wait_gave_up():
     """Tensor-core GEMV launches leave the timeout count where it was."""
     import ctypes
