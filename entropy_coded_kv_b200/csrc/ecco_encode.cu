@@ -19,10 +19,12 @@
 // Selection variants (template SEL, runtime npat): SEL = 1 picks the pattern
 // by the full squared error of the normalised group instead of min/max (the
 // comparison the review page's referee report asks for, major comment 2):
-// each lane quantises its 8 values under every pattern, sums the squared
+// for a pattern it sums, each lane quantises its 8 values, sums the squared
 // errors pairwise and the 16 lanes finish the pairwise tree with xor
 // shuffles (lane l holds slots 8l..8l+7, so the butterfly is the same binary
-// tree over slot order on every lane; fp32 addition is commutative).  npat
+// tree over slot order on every lane; fp32 addition is commutative).  A
+// lower bound from the group's two extreme elements skips the patterns that
+// cannot be the first minimum (encode_group).  npat
 // limits the search to patterns 0..npat-1 (free parameters: 16 patterns in
 // the compressor, "reduced from 64").
 //
@@ -136,6 +138,33 @@ __device__ __forceinline__ int quantise(uint32_t R, float t7, float v)
     return idx;
 }
 
+// The min / max rule's pattern (R8): this lane evaluates patterns hl + kLanes k
+// (those below npat).  e >= +0, so bit order is value order; a pattern past
+// npat gets 0xffffffff, above every error including +inf, so a group whose
+// errors are all +inf still gets the lowest index, as scanning does.
+template <int kLanes>
+__device__ __forceinline__ int minmax_pattern(const DevTables* __restrict__ tb, const float2 (&ends)[4], float umin,
+                                              float umax, int hl, uint32_t gmask, int npat)
+{
+    constexpr int kPatPerLane = kNPat / kLanes;
+    uint32_t eb = 0xffffffffu, bp = 64u;
+#pragma unroll
+    for (int k = 0; k < kPatPerLane; ++k) {
+        const int pat = hl + kLanes * k;
+        // 8 lanes (activation groups) hold 8 patterns each: read from L1 instead of registers
+        const float2 cp = (kPatPerLane <= 4) ? ends[k % 4] : __ldg(&tb->ends[pat]);
+        float d0 = __fsub_rn(umin, cp.x), d1 = __fsub_rn(umax, cp.y);
+        float e = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
+        const uint32_t ek = (pat < npat) ? __float_as_uint(e) : 0xffffffffu;
+        if (ek < eb) {
+            eb = ek;
+            bp = (uint32_t)pat;
+        }
+    }
+    const uint32_t emin = hw_min(gmask, eb);
+    return (int)hw_min(gmask, eb == emin ? bp : 64u);
+}
+
 // Encodes one group of G values with the G/8 lanes of `gmask`; hl = lane
 // within the group.  cent: centroids [64][16] (SEL = 1 only).
 template <int SEL, int G>
@@ -206,36 +235,30 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
         for (int j = 0; j < 8; ++j) e[j] = (j == jm) ? -INFINITY : u[j];
         lmax = fmaxf(fmaxf(fmaxf(e[0], e[1]), fmaxf(e[2], e[3])), fmaxf(fmaxf(e[4], e[5]), fmaxf(e[6], e[7])));
     }
-    int p;
-    if constexpr (SEL == 0) {
-        const float umin = hw_minf(gmask, lmin);
-        const float umax = hw_maxf(gmask, lmax);
-
-        // ---- pattern: this lane evaluates patterns hl + kLanes k (those below
-        // npat).  e >= +0, so bit order is value order; a pattern past npat
-        // gets 0xffffffff, above every error including +inf, so a group whose
-        // errors are all +inf still gets the lowest index, as scanning does.
-        uint32_t eb = 0xffffffffu, bp = 64u;
-#pragma unroll
-        for (int k = 0; k < kPatPerLane; ++k) {
-            const int pat = hl + kLanes * k;
-            // 8 lanes (activation groups) hold 8 patterns each: read from L1 instead of registers
-            const float2 cp = (kPatPerLane <= 4) ? ends[k % 4] : __ldg(&tb->ends[pat]);
-            float d0 = __fsub_rn(umin, cp.x), d1 = __fsub_rn(umax, cp.y);
-            float e = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
-            const uint32_t ek = (pat < npat) ? __float_as_uint(e) : 0xffffffffu;
-            if (ek < eb) {
-                eb = ek;
-                bp = (uint32_t)pat;
-            }
-        }
-        const uint32_t emin = hw_min(gmask, eb);
-        p = (int)hw_min(gmask, eb == emin ? bp : 64u);
-    } else {
-        // ---- pattern by the full squared error (slot m adds +0), scanned in order
-        float best = 0.0f;
-        p = 0;
-        for (int q = 0; q < npat; ++q) {
+    const float umin = hw_minf(gmask, lmin);
+    const float umax = hw_maxf(gmask, lmax);
+    int p = minmax_pattern<kLanes>(tb, ends, umin, umax, hl, gmask, npat);
+    if constexpr (SEL == 1) {
+        // ---- pattern by the full squared error (slot m adds +0): the first
+        // pattern, in index order, with the least error.  An error is a tree
+        // of rounded additions of non-negative terms; rounding is monotone, so
+        // setting every term but two to zero can only lower it, and what is
+        // left is the rounded sum of those two: term(umin) + term(umax) (two
+        // distinct elements other than m, computed with the same operations)
+        // bounds each pattern's error from below.  A pattern whose bound
+        // exceeds the min / max rule's pattern's error cannot be the first
+        // minimum; the others are summed in order, and once one is the best
+        // so far, the later ones whose bound is not below it are dropped too
+        // (a tie goes to the earlier index).
+        auto term = [&](int q, float v) {
+            const uint32_t Rq = (uint32_t)__cvta_generic_to_shared(rows) + (uint32_t)(q * kRow) * 4u;
+            const float4 qmq = qmap[q];
+            const int sq = (qmq.z == 0.0f) ? quantise_bucket(Rq, QL + (uint32_t)q * 256u, qmq, v)
+                                           : quantise(Rq, __uint_as_float(lds_u32(Rq + 28u)), v);
+            const float d = __fsub_rn(v, cent[q * 16 + sq]);
+            return __fmul_rn(d, d);
+        };
+        auto error = [&](int q) {
             const uint32_t Rq = (uint32_t)__cvta_generic_to_shared(rows) + (uint32_t)(q * kRow) * 4u;
             const float* Cq = cent + q * 16;
             const float tq = __uint_as_float(lds_u32(Rq + 28u));
@@ -252,9 +275,36 @@ __device__ __forceinline__ void encode_group(const DevTables* __restrict__ tb, c
                                 __fadd_rn(__fadd_rn(d2[4], d2[5]), __fadd_rn(d2[6], d2[7])));
 #pragma unroll
             for (int o = 1; o < kLanes; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(gmask, v, o));
-            if (q == 0 || v < best) {
+            return v;
+        };
+        const float known = error(p);
+        const int base = __ffs(gmask) - 1;  // the group's first lane in the warp
+        float lb[kPatPerLane];              // bounds of this lane's patterns hl + kLanes k
+        uint64_t keep = 0;                  // bit q: pattern q may be the first minimum
+#pragma unroll
+        for (int k = 0; k < kPatPerLane; ++k) {
+            const int pat = hl + kLanes * k;
+            lb[k] = (pat < npat) ? __fadd_rn(term(pat, umin), term(pat, umax)) : __int_as_float(0x7f800000);
+            const bool may = pat < npat && !(lb[k] > known);
+            const uint32_t bits = (__ballot_sync(gmask, may) >> base) & ((1u << kLanes) - 1u);
+            keep |= (uint64_t)bits << (kLanes * k);
+        }
+        float best = 0.0f;
+        p = -1;
+        while (keep) {  // uniform in the group
+            const int q = __ffsll((long long)keep) - 1;
+            keep &= keep - 1;
+            const float v = error(q);
+            if (p < 0 || v < best) {
                 best = v;
                 p = q;
+                uint64_t below = 0;  // the patterns whose bound is below the new best
+#pragma unroll
+                for (int k = 0; k < kPatPerLane; ++k) {
+                    const uint32_t bits = (__ballot_sync(gmask, lb[k] < best) >> base) & ((1u << kLanes) - 1u);
+                    below |= (uint64_t)bits << (kLanes * k);
+                }
+                keep &= below;
             }
         }
     }

@@ -134,7 +134,7 @@ int ecco_select_encode(const ecco_tables* tables, const uint16_t* x_bf16, ecco_d
  *                       fp32 sum of (u_i - C[p][sym_p(u_i)])^2, the scale
  *                       element adding 0; first p with the least e_p.  The
  *                       comparison the review page's referee report asks for
- *                       (major comment 2); about 10x the encoder's work.
+ *                       (major comment 2); about 6x the encoder's time.
  * `n_patterns` (1..64): only patterns 0..n_patterns-1 are searched (free
  * parameters: the compressor's 16 patterns, "reduced from 64"); tables for it
  * are learned with that many patterns.  Blocks decode with ecco_decode as
