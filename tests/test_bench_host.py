@@ -97,3 +97,22 @@ def test_reference_arm_runs_the_oracle_alone(workload):
     if want is not bench.AttnWorkload:
         assert line["config"]["workload"] == want.desc
     assert out[-1] == "LIBS 0 1"
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_0():
+    """Launched the way the scaling run launches it (torchrun, 2 ranks, gloo
+    on the host): rank 0 alone times the oracle and prints, the other rank
+    exits 0, and the line counts both ranks."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--workload", "c1", "--steps", "1", "--warmup", "1"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
