@@ -63,12 +63,22 @@ def parse_args():
 
 
 def peaks():
+    """HBM copy bandwidth (GB/s) from MEASURED_PEAKS.json's hbm_gbs (a number,
+    or an object holding one under value / gbs / burst), else the fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+    if not os.path.exists(p):
+        return FALLBACK_HBM_GBS, "fallback"
+    try:
         with open(p) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+            v = json.load(f)["hbm_gbs"]
+        if isinstance(v, dict):
+            v = next(v[k] for k in ("value", "gbs", "burst") if k in v)
+        v = float(v)
+        if v > 0:
+            return v, "measured"
+    except (OSError, ValueError, KeyError, TypeError, StopIteration):
+        pass
+    return FALLBACK_HBM_GBS, "fallback (MEASURED_PEAKS.json has no usable hbm_gbs)"
 
 
 # ------------------------------------------------------------------ clocks

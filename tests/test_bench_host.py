@@ -59,6 +59,23 @@ def test_source_hash_covers_every_listed_file():
         assert len(bench.source_hash(files)) == 16
 
 
+@pytest.mark.parametrize("content,want", [
+    ('{"hbm_gbs": 6532.5}', (6532.5, "measured")),
+    ('{"hbm_gbs": {"value": 6400}}', (6400.0, "measured")),
+    ('{"bf16_tflops": 1500}', None),
+    ('{"hbm_gbs": "n/a"}', None),
+    ('not json', None),
+])
+def test_peak_file_forms(tmp_path, monkeypatch, content, want):
+    (tmp_path / "MEASURED_PEAKS.json").write_text(content)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    value, source = bench.peaks()
+    if want is None:
+        assert value == bench.FALLBACK_HBM_GBS and source.startswith("fallback")
+    else:
+        assert (value, source) == want
+
+
 def test_peak_comes_from_the_measured_file_when_present():
     value, source = bench.peaks()
     if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
