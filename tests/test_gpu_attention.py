@@ -163,6 +163,33 @@ def test_full_size_kv_cache_attention_sampled():
         check(outs[b:b + 1, h * G:(h + 1) * G], ref, aw)
 
 
+def test_long_context_layer_attention_sampled():
+    """One long-context layer, K and V [1, 8, 131072, 128], 32 query heads:
+    the merge combines 256 splits (fused) and 512 (staged) per head.  Two KV
+    heads against the oracle, whose blocks are its own encoding."""
+    K, V = W.c5_layer(0, device=DEV)
+    Kc, Vc = W.c5_calibration(0, device=DEV)
+    kt, vt = learn_tables(Kc, seed=0), learn_tables(Vc, seed=0)
+    tk, tv = ecco.Tables(kt, DEV), ecco.Tables(vt, DEV)
+    B, H, S, _ = K.shape
+    G = 4
+    kb = ecco.encode(K, tk).view(B, H, S, 64)
+    vb = ecco.encode(V, tv).view(B, H, S, 64)
+    q = q_bits(B, H * G, seed=41)
+    scale = 1.0 / np.sqrt(128.0)
+    out = ecco.decode_attention(kb, vb, tk, tv, to_dev_bf16(q), S, scale).cpu().numpy()
+    outs = ecco.decode_attention_staged(kb, vb, tk, tv, to_dev_bf16(q), S, scale).cpu().numpy()
+    for h in (0, 6):
+        kbo, _ = oracle.encode(kt, W.bf16_bits(K[0, h]), nthreads=8)
+        vbo, _ = oracle.encode(vt, W.bf16_bits(V[0, h]), nthreads=8)
+        np.testing.assert_array_equal(kb[0, h].cpu().numpy(), kbo)
+        np.testing.assert_array_equal(vb[0, h].cpu().numpy(), vbo)
+        ref, aw = oracle.attention(kt, vt, kbo.reshape(1, 1, S, 64), vbo.reshape(1, 1, S, 64),
+                                   q[:, h * G:(h + 1) * G], S, scale, nthreads=8)
+        check(out[:, h * G:(h + 1) * G], ref, aw)
+        check(outs[:, h * G:(h + 1) * G], ref, aw)
+
+
 def test_attention_argument_errors():
     lib = _lib.load()
     t = ecco.Tables(table_set("learned_kv"), DEV)
