@@ -13,7 +13,8 @@
 // accumulators.  When the units do not divide evenly over the CTAs and the
 // remainder is small, the remainder is not handed out whole (one more round
 // on a few SMs, the rest idle): its units are cut into warp steps of 32 rows,
-// which every CTA's first warps take after their whole units.  Thread t decodes row t's block of the unit with the block
+// spread over the CTAs, and in each CTA the warps that finish their whole
+// units first claim them.  Thread t decodes row t's block of the unit with the block
 // walker of ecco_block.cuh.  The walk's speed comes from the warps running
 // freely (its latency is hidden by the other warps), so every warp feeds the
 // tensor cores on its own, with no barrier between warps inside a unit:
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     uint8_t* s_B = smem + kOffB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
+    unsigned int* s_next = reinterpret_cast<unsigned int*>(s_tmem + 1);  // leftover steps claimed so far
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = warp >> 2;               // 4 warps per 128-row tile
@@ -200,6 +202,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     uint64_t* bar_full = &bars[2 * kTcWarps];
     uint64_t* bar_free = &bars[2 * kTcWarps + kBSlots];
     if (tid == 0) {
+        *s_next = 0u;
         for (int i = 0; i < 2 * kTcWarps; ++i) mbar_init(&bars[i], 1);
         for (int i = 0; i < kBSlots; ++i) {
             mbar_init(&bar_full[i], kTcThreads);  // every thread writes a share of x
@@ -407,10 +410,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     }
     flush(tile_row, warp * 32);
 
-    // The CTA's leftover steps: warp w takes step ts0 + w (32 rows of a
-    // leftover unit), with the SM nearly to itself.
-    if (warp < ts1 - ts0) {
-        const int64_t j = ts0 + warp, tu = j / kTcWarps;
+    // The CTA's leftover steps (32 rows of a leftover unit each), claimed one
+    // at a time by the warps that finish their units first, while the others
+    // are still on their last.
+    for (;;) {
+        unsigned int c = 0;
+        if (lane == 0) c = atomicAdd(s_next, 1u);
+        c = __shfl_sync(0xffffffffu, c, 0);
+        if ((int64_t)c >= ts1 - ts0) break;
+        const int64_t j = ts0 + (int64_t)c, tu = j / kTcWarps;
         const int64_t u = A.units + tu, rt = u / A.gpr, g = u - rt * A.gpr;
         const int rb = (int)(j - tu * kTcWarps) * 32;
         run_unit(nu + (tu - tl0), rt, g, rb);
