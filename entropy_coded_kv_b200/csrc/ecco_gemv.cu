@@ -7,11 +7,12 @@
 //
 // Layout of the work: an item is one strip of 32 rows (a warp, a lane per
 // row) x one column group, numbered column group by column group.  Each CTA
-// (one per SM, resident) owns a balanced, contiguous range of items and runs
-// it in rounds of one item per warp, so CTAs differ by at most one item and
-// a CTA's last round is short (whole units of one row per thread would leave
+// (one per SM, resident) owns a balanced, contiguous range of items, so CTAs
+// differ by at most one item (whole units of one row per thread would leave
 // the SMs that own one unit fewer idle for a quarter of the launch at the
-// 14336 x 4096 shape).  All lanes of a warp need the same x[k] at every step
+// 14336 x 4096 shape).  When the range lies in one x window its warps claim
+// items from a shared counter as they finish; otherwise they run it in rounds
+// of one item per warp.  All lanes of a warp need the same x[k] at every step
 // (a broadcast shared-memory read); x is staged in windows of 32 column
 // groups, restaged when a round reaches past the window.  Each lane decodes
 // its row's block serially (one lookup per symbol, as in the decoder) and
@@ -70,22 +71,9 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
     uint32_t* nibs = s_nib + tid;
     int64_t win0 = -1;  // first column group of the staged x window
 
-    for (int64_t q0 = qa; q0 < qb; q0 += kWarps) {
-        // the round's column groups must lie in the window (uniform across the CTA)
-        const int64_t g_first = q0 / strips, g_last = (min(q0 + kWarps, qb) - 1) / strips;
-        if (win0 < 0 || g_first < win0 || g_last >= win0 + kGvWin) {
-            __syncthreads();  // the previous window is no longer read (and the tables are staged)
-            win0 = g_first;
-            const int64_t k0 = win0 * kG;
-            const int nk = (int)min((int64_t)kGvWin * kG, cols - k0);
-            for (int i = tid; i < kGvWin * kG * B; i += kGvThreads) {
-                const int k = i / B, bb = i - k * B;
-                s_x[i] = (bb < batch && k < nk) ? bf16_bits_to_f32(x[(int64_t)bb * cols + k0 + k]) : 0.0f;
-            }
-            __syncthreads();
-        }
-        const int64_t q = q0 + warp;
-        if (q >= qb) continue;  // this warp has no item in the CTA's short last round
+    // One item: this warp's 32 rows of column group q / strips, x from the
+    // staged window.
+    auto do_item = [&](int64_t q) {
         const int64_t gcol = q / strips;
         const int64_t row = (q - gcol * strips) * 32 + lane;
         const bool row_ok = row < rows;
@@ -166,6 +154,50 @@ __global__ void __launch_bounds__(gv_threads<B>(), 1)
             for (int bb = 0; bb < B; ++bb)
                 if (bb < batch) atomicAdd(&y[(int64_t)bb * rows + row], acc[bb]);
         }
+    };
+
+    __shared__ unsigned int s_next;  // items of the CTA's range claimed so far
+    if (qb > qa && (qb - 1) / strips - qa / strips < kGvWin) {
+        // The whole range lies in one x window: staged once, and the warps
+        // claim items one at a time as they finish, so the range's last items
+        // go to the warps that are free first, not to fixed warps in a short
+        // last round.
+        const int64_t k0 = (qa / strips) * kG;
+        const int nk = (int)min((int64_t)kGvWin * kG, cols - k0);
+        for (int i = tid; i < kGvWin * kG * B; i += kGvThreads) {
+            const int k = i / B, bb = i - k * B;
+            s_x[i] = (bb < batch && k < nk) ? bf16_bits_to_f32(x[(int64_t)bb * cols + k0 + k]) : 0.0f;
+        }
+        win0 = qa / strips;
+        if (tid == 0) s_next = 0u;
+        __syncthreads();  // window, tables and counter ready
+        for (;;) {
+            unsigned int c = 0;
+            if (lane == 0) c = atomicAdd(&s_next, 1u);
+            c = __shfl_sync(0xffffffffu, c, 0);
+            if (qa + (int64_t)c >= qb) break;
+            do_item(qa + (int64_t)c);
+        }
+        return;
+    }
+
+    for (int64_t q0 = qa; q0 < qb; q0 += kWarps) {
+        // the round's column groups must lie in the window (uniform across the CTA)
+        const int64_t g_first = q0 / strips, g_last = (min(q0 + kWarps, qb) - 1) / strips;
+        if (win0 < 0 || g_first < win0 || g_last >= win0 + kGvWin) {
+            __syncthreads();  // the previous window is no longer read (and the tables are staged)
+            win0 = g_first;
+            const int64_t k0 = win0 * kG;
+            const int nk = (int)min((int64_t)kGvWin * kG, cols - k0);
+            for (int i = tid; i < kGvWin * kG * B; i += kGvThreads) {
+                const int k = i / B, bb = i - k * B;
+                s_x[i] = (bb < batch && k < nk) ? bf16_bits_to_f32(x[(int64_t)bb * cols + k0 + k]) : 0.0f;
+            }
+            __syncthreads();
+        }
+        const int64_t q = q0 + warp;
+        if (q >= qb) continue;  // this warp has no item in the CTA's short last round
+        do_item(q);
     }
 }
 
