@@ -280,6 +280,21 @@ def test_gemv_within_tolerance(batch, rows, cols):
     gemv_check(blob, blocks, rows, cols, xb, y)
 
 
+@pytest.mark.parametrize("batch", [1, 3])
+def test_gemv_restages_x_windows(batch):
+    """A matrix so wide (5,000 column groups, one strip of rows) that a CTA's
+    items span more than one 32-group window of x: the CUDA-core product runs
+    its items in rounds and restages x as they move on."""
+    blob = table_set("learned_w")
+    rows, cols = 7, 128 * 5000
+    wb = inputs("t5", rows * cols // 128, seed=12)
+    blocks, _ = oracle.encode(blob, wb, nthreads=8)
+    t = ecco.Tables(blob, DEV)
+    xb = bits(torch.randn(batch, cols, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16))
+    y = ecco.decode_gemv(torch.from_numpy(blocks).to(DEV), t, rows, cols, to_dev_bf16(xb)).cpu().numpy()
+    gemv_check(blob, blocks, rows, cols, xb, y)
+
+
 def test_gemv_one_hot_selects_a_decoded_column_exactly():
     blob = table_set("learned_w")
     rows, cols = 300, 256
